@@ -1,0 +1,88 @@
+"""Seeded synthetic inputs for the mixer stack.
+
+This module holds no arithmetic of the method itself: it only draws filters and
+input tokens.  Both the CUDA path's callers (tests, bench) and the CPU oracle are
+fed the same arrays from here, so the choice of generator can never cause a
+mismatch between the two.
+
+Recipe (random-init weights, as in the experimental setup of the Flash Inference
+paper summary, section "Experimentelle Einrichtung"):
+
+* filter of layer l, channel c, tap k:
+  ``h[l, c, k] = N(0,1) * exp(-a_c * k) / sqrt(32)`` with ``a_c ~ U(0.001, 0.05)``;
+  every layer draws its own ``a`` and its own normals ("same law", not the same draw).
+* inputs: ``x ~ N(0,1)`` i.i.d. over (t, b, c); closed loop starts from one
+  ``x_0 ~ N(0,1)`` per (b, c).
+
+Generator: numpy PCG64 seeded through ``SeedSequence([seed, stream, l])``, one
+independent stream per layer (stream 1), one for teacher-forced inputs (stream 2)
+and one for the closed-loop start token (stream 3).  Within a layer stream the
+draw order is: ``a_c`` for all c, then the normals in [c][k] order.
+"""
+from __future__ import annotations
+
+import math
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+A_LO, A_HI = 0.001, 0.05
+SCALE = 1.0 / math.sqrt(32.0)
+
+
+def _rng(seed: int, stream: int, sub: int = 0) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, stream, sub])))
+
+
+def _layer(out: np.ndarray, seed: int, l: int, decay: bool, chunk: int = 64) -> None:
+    D, L = out.shape
+    g = _rng(seed, 1, l)
+    a = g.uniform(A_LO, A_HI, size=D)
+    if not decay:
+        a[:] = 0.0
+    k = np.arange(L, dtype=np.float64)
+    for c0 in range(0, D, chunk):
+        c1 = min(D, c0 + chunk)
+        z = g.standard_normal((c1 - c0, L))
+        z *= np.exp(-a[c0:c1, None] * k[None, :])
+        z *= SCALE
+        out[c0:c1] = z
+
+
+def filters(M: int, D: int, L: int, seed: int = 0, decay: bool = True,
+            threads: int | None = None, out: np.ndarray | None = None) -> np.ndarray:
+    """float32 [M][D][L] decaying-exponential random filters (one stream per layer).
+
+    ``decay=False`` keeps the same normals but sets every ``a_c`` to 0, giving
+    non-decaying filters whose long lags are not negligible (used to exercise
+    the large tiles numerically)."""
+    h = np.empty((M, D, L), np.float32) if out is None else out
+    assert h.shape == (M, D, L) and h.dtype == np.float32
+    if threads is None:
+        import os
+        threads = min(M, max(1, len(os.sched_getaffinity(0))))
+    if threads <= 1 or M == 1:
+        for l in range(M):
+            _layer(h[l], seed, l, decay)
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda l: _layer(h[l], seed, l, decay), range(M)))
+    return h
+
+
+def inputs(T: int, B: int, D: int, seed: int = 0) -> np.ndarray:
+    """float32 [T][B][D] teacher-forced tokens, N(0,1)."""
+    return _rng(seed, 2).standard_normal((T, B, D)).astype(np.float32)
+
+
+def start_token(B: int, D: int, seed: int = 0) -> np.ndarray:
+    """float32 [B][D] closed-loop start token x_0, N(0,1)."""
+    return _rng(seed, 3).standard_normal((B, D)).astype(np.float32)
+
+
+# Workloads (layers, B, D, L) of the measured configurations.
+CONFIGS = {
+    "tiny": dict(M=1, B=1, D=16, L=1 << 10),
+    "headline": dict(M=18, B=1, D=864, L=1 << 17),
+    "hyena_shape": dict(M=18, B=4, D=768, L=1 << 15),
+}
