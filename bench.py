@@ -1,0 +1,384 @@
+"""Benchmark: closed-loop generation through the mixer stack (mixer tokens/s).
+
+One "step" = one whole L-token closed-loop generation (fi_reset + fi_generate from
+t = 0) of the stack of 18 long-convolution layers, B=1, D=864, L=2^17, fp32,
+synthetic seeded filters: every block, red cell, sampler and tanh of the path runs
+inside it.  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank generates its own sequence
+(independent start token) with the same model; no data-path collective.  Weak
+scaling; value = all ranks' tokens / max-over-ranks time.
+--impl reference times the CPU oracle (plain fp64 lazy evaluation) on the host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "mixer tokens/s (B·L/time) at 18L×D864×L=2^17; % of HBM/fp32 roofline"
+WORKLOADS = {
+    # name: (layers, B, D, L)
+    "headline": (18, 1, 864, 1 << 17),
+    "hyena_shape": (18, 4, 768, 1 << 15),
+    "tiny": (1, 1, 16, 1 << 10),
+}
+FALLBACK_HBM_GBS = 6650.0
+FP32_LANES_PER_SM = 128
+
+
+# ------------------------------------------------------------------ cost model
+def model_bytes_flops(M, B, D, L):
+    """Algorithmic work of one L-token generation (whole stack).
+
+    Per (layer, channel) and tile of edge U: block read B*U, output read-modify-write
+    2*B*U, taps or spectrum 2U (shared over the batch), all fp32; per token the red
+    cell reads/writes 2B+1 values.  FLOPs per tile and batch row: the cheaper of the
+    direct 2U^2 and two real 2U-point FFTs (2.5 N log2 N each) + complex product +
+    accumulate; per token 2 flops of red cell."""
+    P = L.bit_length() - 1
+    byts = 0
+    flops = 0
+    for q in range(P):
+        U = 1 << q
+        ntile = 1 << (P - 1 - q)
+        byts += ntile * 4 * (3 * B * U + 2 * U)
+        flops += ntile * B * min(2 * U * U, 10 * U * math.log2(2 * U) + 6 * (U + 1) + U)
+    byts += L * 4 * (2 * B + 1)
+    flops += B * 2 * L
+    return byts * M * D, flops * M * D
+
+
+def level_bytes(M, B, D, L, q):
+    """Algorithmic bytes of one launch of the blocks of edge 2^q (all layers/channels)."""
+    U = 1 << q
+    return M * D * 4 * (3 * B * U + 2 * U)
+
+
+def window_bytes(M, B, D, L, W):
+    """Algorithmic bytes of one window-kernel launch: W tokens of red cells plus every
+    block of edge < W released inside the window (same per-tile model)."""
+    w = W.bit_length() - 1
+    per_token = w * 2 * (3 * B + 2) + 4 * (2 * B + 1)
+    return M * D * W * per_token
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        mhz = d.get("sm_max_mhz", 1965.0)
+        return d["hbm_gbs"], "measured", mhz
+    return FALLBACK_HBM_GBS, "fallback", 1965.0
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = Path("/tmp/fi_bench_clocks_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in self.path.read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        self.path.unlink(missing_ok=True)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(h, x0, T_s, G_s, M, B, D, L):
+    """Time the fp64 lazy oracle on G_s chains (channels 0..G_s-1 of batch row 0), all
+    layers, the first T_s closed-loop tokens; return (tokens/s for the whole workload,
+    seconds, description).  The lazy oracle's work is M * chains * T(T+1)/2 MACs, so
+    the whole-workload time is the measured time scaled by that count."""
+    import oracle
+    hs = np.ascontiguousarray(h[:, :G_s, :T_s])
+    xs = np.ascontiguousarray(x0[:1, :G_s])
+    t0 = time.perf_counter()
+    oracle.stack(hs, xs, T=T_s, closed_loop=True, want=("y_last",))
+    sec = time.perf_counter() - t0
+    full = sec * (B * D / G_s) * (L * (L + 1) / 2) / (T_s * (T_s + 1) / 2)
+    desc = ("%d chains x %d layers x first %d of %d tokens, closed loop; time scaled by chains "
+            "(x%g) and by the lazy cost T(T+1)/2 (x%.1f)" % (G_s, M, T_s, L, B * D / G_s,
+                                                            (L * (L + 1)) / (T_s * (T_s + 1))))
+    return B * L / full, sec, desc
+
+
+def oracle_sample_size(M, L, budget_s=15.0, rate=1.0e9):
+    T_s = int(math.sqrt(2 * budget_s * rate / M))
+    T_s = 1 << max(8, min(L.bit_length() - 1, T_s.bit_length() - 1))
+    return min(T_s, L)
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="headline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-trace", action="store_true", help="do not bracket launches with events")
+    ap.add_argument("--path", choices=("window", "token"), default="window")
+    ap.add_argument("--graphs", type=int, default=1)
+    args = ap.parse_args()
+    M, B, D, L = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from long_convolution_sequence_b200 import synth
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return bench_reference(args, M, B, D, L, synth)
+
+    import torch
+    import torch.distributed as dist
+    import datetime
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    import long_convolution_sequence_b200 as fi
+
+    t_setup = time.perf_counter()
+    h = synth.filters(M, D, L, seed=0)
+    x0 = synth.start_token(B, D, seed=rank)
+    t_gen = time.perf_counter() - t_setup
+    t0 = time.perf_counter()
+    ctx = fi.FlashInference(M, B, D, L, h)
+    t_create = time.perf_counter() - t0
+    ctx.set_path(fi.FI_PATH_WINDOW if args.path == "window" else fi.FI_PATH_TOKEN)
+    ctx.set_graphs(bool(args.graphs))
+    trace = not args.no_trace
+    ctx.set_trace(trace)
+    info = ctx.info()
+
+    x0_d = torch.from_numpy(x0).cuda()
+    out_d = torch.empty((L, B, D), device="cuda")
+
+    def one_step():
+        ctx.reset()
+        ctx.generate(x0_d, L, out_d)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+
+    clocks = Clocks(local)
+    launches0 = ctx.info().launches
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        one_step()
+    ev1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    launches = ctx.info().launches - launches0
+    tr = ctx.trace() if trace else {}
+    if world > 1:
+        tms = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
+        ms = float(tms.item())
+
+    # end to end through the public API: host (pinned) start token in, host result out
+    x0_h = torch.from_numpy(x0).pin_memory()
+    out_h = torch.empty((L, B, D), pin_memory=True)
+    ctx.set_trace(False)
+    ctx.reset()
+    ctx.generate(x0_h, L, out_h)  # capture / warm
+    e2e_steps = max(1, min(args.steps, 3))
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        ctx.reset()
+        ctx.generate(x0_h, L, out_h)
+    e2e_sec = (time.perf_counter() - t0) / e2e_steps
+    if world > 1:
+        te = torch.tensor([e2e_sec], device="cuda")
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_sec = float(te.item())
+    finite = bool(np.isfinite(out_h.numpy()).all())
+
+    if rank != 0:
+        ctx.close()
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    hbm, peak_kind, sm_mhz = peaks()
+    tokens = world * B * L
+    value = tokens / (ms / 1000.0)
+    byts, flops = model_bytes_flops(M, B, D, L)
+    fp32_peak = info.sm_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6
+    t_roof = max(byts / (hbm * 1e9), flops / fp32_peak)
+
+    roof = None
+    if tr:
+        dom = max(tr, key=lambda k: tr[k][1])
+        n_l, tot_us, max_us = tr[dom]
+        avg_s = tot_us / n_l * 1e-6
+        if dom == "window":
+            per_launch = window_bytes(M, B, D, L, info.window)
+            unit_desc = "W=%d tokens x (red cells + blocks of edge < W), %d layers x %d channels" % (
+                info.window, M, D)
+        else:
+            per_launch = byts / max(1, n_l)
+            unit_desc = "mean block launch"
+        ach = per_launch / avg_s / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 4), "traffic": None, "kernel": dom,
+                "launches_per_step": n_l, "avg_launch_us": round(tot_us / n_l, 2),
+                "bytes_per_launch": per_launch, "per_launch_work": unit_desc,
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                else "fallback 6.65 TB/s"}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+        T_s = oracle_sample_size(M, L)
+        G_s = min(B * D, max(1, oracle.num_threads()))
+        val, sec, desc = time_oracle(h, x0, T_s, G_s, M, B, D, L)
+        cpu = {"value": round(val, 3), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+               "sample": desc, "sample_seconds": round(sec, 2)}
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic: seeded decaying-exponential random filters, N(0,1) start token",
+        "config": {"workload": "closed-loop generation of %d tokens through %d long-convolution layers, "
+                               "B=%d, D=%d, tanh block and sampler" % (L, M, B, D),
+                   "layers": M, "B": B, "D": D, "L": L, "window": info.window,
+                   "path": args.path, "graphs": bool(args.graphs),
+                   "tau": {str(q): ("fft" if info.tau[q] == fi.FI_TAU_FFT else "direct")
+                           for q in range(L.bit_length() - 1)},
+                   "l2": "inputs larger than L2: %.1f GB of buffers, filters and spectra resident per GPU"
+                         % (info.device_bytes / 1e9),
+                   "parallelism": "replicas x%d (one sequence per GPU)" % world},
+        "e2e": {"value": round(tokens / e2e_sec, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": B * D * 4, "d2h_bytes_per_step": L * B * D * 4},
+        "gpu_launches": int(launches),
+        "roofline": roof,
+        "job_roofline": {"model_bytes": byts, "model_flops": flops, "t_roof_ms": round(t_roof * 1e3, 3),
+                         "frac": round(t_roof * 1e3 / ms, 4), "hbm_gbs": hbm,
+                         "fp32_tflops": round(fp32_peak / 1e12, 1),
+                         "note": "time of the slower of model bytes at HBM peak and model FLOPs at fp32 peak, "
+                                 "divided by the measured step time"},
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "kernel_time_us": {k: round(v[1], 1) for k, v in tr.items()},
+        "setup_s": {"filters": round(t_gen, 2), "create": round(t_create, 2)},
+        "outputs_finite": finite,
+        "context": "pages' figures (H100/A100, precision not stated): 110x mixer and 7.8x end-to-end "
+                   "speedup over lazy inference",
+    }
+    print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_reference(args, M, B, D, L, synth):
+    """The oracle as the reference arm: each step times a bounded sample of the same
+    workload on the host cores and scales it to the metric's unit."""
+    import oracle
+    T_s = oracle_sample_size(M, L, budget_s=max(3.0, 60.0 / max(1, args.steps + args.warmup)))
+    G_s = min(B * D, max(1, oracle.num_threads()))
+    hs = np.ascontiguousarray(synth.filters(M, G_s, T_s, seed=0))
+    x0 = synth.start_token(B, D, seed=0)
+    for _ in range(args.warmup):
+        time_oracle(hs, x0, min(T_s, 1024), G_s, M, B, D, L)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, s, desc = time_oracle(hs, x0, T_s, G_s, M, B, D, L)
+        vals.append(v)
+        secs.append(s)
+    value = len(vals) / sum(1.0 / v for v in vals)
+    ms = B * L / value * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded decaying-exponential random filters, N(0,1) start token",
+        "config": {"workload": "closed-loop generation of %d tokens through %d long-convolution layers, "
+                               "B=%d, D=%d, tanh block and sampler" % (L, M, B, D),
+                   "layers": M, "B": B, "D": D, "L": L},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,190 @@
+/*
+ * fi.h -- C-ABI of the B200 Flash Inference mixer library (libfi.so).
+ *
+ * The library runs exact autoregressive inference of a stack of long causal
+ * convolutions ("LCSM" mixers), one filter per layer and channel, with the
+ * relaxed power-of-two tiling of the Flash Inference paper.  Citations below
+ * name the web summary of arXiv 2410.12982, "Flash Inference: Near Linear Time
+ * Inference for Long Convolution Sequence Models and Beyond", by section:
+ *
+ *   [Def]   section "LCSM-spezifische Definition":
+ *           mixer^l(y)_t = sum_{i<=t} y_i (.) rho^l_{t-i}  (per channel, depthwise)
+ *   [Alg1]  section "Kachelung-Strategie (Algorithmus 1)": after token i, with U the
+ *           largest power of two dividing i, the red cell z_i += y_i rho_0 and the
+ *           gray block z[i+1 .. i+U] += tau(y, [i-U+1, i], rho, [i+1, i+U])
+ *   [Alg2]  section "LCSM-Inferenz-Algorithmus (Algorithmus 2)": the same over M
+ *           layers, a^l_i = block^l(b^l_i), a^0_{i+1} = sampler(a^M_i)
+ *   [Alg3]  section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)": red
+ *           cells in layer order, the gray blocks of all layers in parallel
+ *   [Mem]   section "Speicheroptimierung": a^l_i reuses the storage of b^l_i; the
+ *           DFT of the filters is precomputed per block size
+ *   [Circ]  section "Zirkulaere Faltungs-Trick": a 2U circular convolution suffices
+ *   [Impl]  section "Implementierungsdetails": CUDA graphs per token, FFT precompute,
+ *           Hybrid choice of the tau implementation by block size
+ *   [Lem1]  section "Beitrags-Aggregations-Definition", Lemma 1:
+ *           tau(y,[l,r],rho,[l',r'])_t = sum_{i=l}^{r} y_i rho_{t-i}
+ *
+ * Model computed (block^l = tanh, sampler = tanh):
+ *   y^l_t = sum_{s<=t} h^l[c][t-s] * a^{l-1}_s[b][c],   a^l_t = tanh(y^l_t),
+ *   a^0_t = x_t (teacher-forced) or a^0_{t+1} = a^M_t (closed loop).
+ * Positions t are 0-based; the pages' loop counter i is n = t + 1.
+ *
+ * Conventions for every entry point:
+ *   - Arrays are fp32, row-major.  A "chain" is one (b, c) pair, index g = b*D + c.
+ *   - Per-token arrays are [B][D]; sequences are [steps][B][D] (time-major).
+ *   - Pointers may be host or device memory unless stated otherwise; the library
+ *     detects which (cudaPointerGetAttributes).  Calls with host destinations
+ *     return after the data has arrived; calls with device destinations are
+ *     asynchronous on the context's stream.
+ *   - The library never takes ownership of, frees or retains caller memory.
+ *   - Return values: FI_OK (0) or a negative FI_E* code; the message of the last
+ *     failure on the calling thread is available from fi_last_error().
+ *   - A context is not thread-safe; distinct contexts are independent.
+ */
+#ifndef FI_H_
+#define FI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FI_OK 0
+#define FI_EINVAL (-1)      /* bad argument: dims, L not a power of two, null pointer */
+#define FI_ECAPACITY (-2)   /* the call would run past position L-1 */
+#define FI_ENOMEM (-3)      /* device or host allocation failed */
+#define FI_ECUDA (-4)       /* a CUDA call failed; message carries cudaGetErrorString */
+#define FI_ESTATE (-5)      /* null or destroyed context */
+
+/* tau implementations ([Impl] Hybrid) */
+#define FI_TAU_AUTO 0       /* measured choice per block size (the Hybrid scheme) */
+#define FI_TAU_DIRECT 1     /* direct convolution of the block, U^2 multiply-adds */
+#define FI_TAU_FFT 2        /* FFT of the 2U circular convolution against a precomputed
+                               filter spectrum ([Circ], [Mem]) */
+
+/* execution paths of a generation */
+#define FI_PATH_WINDOW 0    /* default: one persistent kernel per aligned window of W
+                               tokens (red cells + all blocks smaller than W, in shared
+                               memory), one launch per larger block */
+#define FI_PATH_TOKEN 1     /* the pages' design: one launch sequence (graph) per token */
+
+typedef struct fi_ctx fi_ctx;
+
+typedef struct fi_info {
+    int layers, B, D, L;        /* as created */
+    int t;                      /* tokens processed so far (next position) */
+    int window;                 /* W of the window path */
+    int chains_per_cta;         /* chains held by one CTA of the window kernel */
+    int path;                   /* FI_PATH_* in use */
+    int graphs;                 /* 1 if launches are replayed from captured CUDA graphs */
+    int tau[32];                /* FI_TAU_DIRECT / FI_TAU_FFT chosen for block size 2^q */
+    float tau_us[32][2];        /* measured microseconds per launch [q][direct, fft]; 0 = not timed */
+    size_t device_bytes;        /* device memory held by the context */
+    int sm_count;               /* SMs of the device */
+    long long launches;         /* kernels launched by this context's runs so far */
+} fi_info;
+
+/* kernel classes reported by fi_trace_read */
+#define FI_K_WINDOW 0        /* window kernel: red cells + blocks smaller than W */
+#define FI_K_TOKEN_STEP 1    /* per-token step kernel: red cells (+ small blocks) */
+#define FI_K_BLOCK_DIRECT 2  /* one block size, every layer and chain, direct tau */
+#define FI_K_BLOCK_FFT 3     /* one block size, every layer and chain, fused FFT tau */
+#define FI_K_BLOCK_SPLIT 4   /* blocks larger than one CTA's FFT, split FFT tau */
+#define FI_K_CLASSES 5
+
+typedef struct fi_trace {
+    int launches[FI_K_CLASSES];     /* launches of each class in the last run */
+    double total_us[FI_K_CLASSES];  /* summed device time of those launches */
+    double max_us[FI_K_CLASSES];    /* longest single launch */
+} fi_trace;
+
+/* Create a context for `layers` stacked mixers over B sequences of D channels,
+ * capacity L positions.  filters: [layers][D][L] fp32 (host or device), filter of
+ * layer l (0-based), channel c, lag k at filters[(l*D + c)*L + k] ([Def]).  The
+ * filters are copied; the caller keeps ownership.  L must be a power of two >= 2.
+ * Precomputes the filter spectra for every block size served by FFT ([Mem]) and
+ * measures the tau choice per block size ([Impl] Hybrid).  Returns NULL on error
+ * (see fi_last_error).  The context starts at t = 0. */
+fi_ctx *fi_create(int layers, int B, int D, int L, const float *filters);
+
+/* Release every resource of the context.  NULL is accepted. */
+void fi_destroy(fi_ctx *ctx);
+
+/* Teacher-forced single token ([Alg2] one loop iteration): x_t [B][D] is token t
+ * (t = the context's counter); y_t [B][D] receives y^M_t, the last layer's mixer
+ * output before tanh.  Afterwards every gray block released by this token has been
+ * applied and t advances by one.  FI_ECAPACITY if t == L. */
+int fi_step(fi_ctx *ctx, const float *x_t, float *y_t);
+
+/* Closed-loop generation of `steps` tokens from the current position t
+ * ([Alg2], sampler = tanh): x0 [B][D] is token t, or NULL to continue from the
+ * token the previous closed-loop call produced (a^M_{t-1}).  out [steps][B][D]
+ * receives y^M_t .. y^M_{t+steps-1}; token t+1 = tanh(y^M_t) stays on the device.
+ * FI_ECAPACITY if t + steps > L.  steps == 0 is a no-op. */
+int fi_generate(fi_ctx *ctx, const float *x0, int steps, float *out);
+
+/* Teacher-forced run over `steps` tokens (the windowed form of fi_step):
+ * x [steps][B][D] are tokens t .. t+steps-1, y [steps][B][D] receives y^M. */
+int fi_forward(fi_ctx *ctx, const float *x, int steps, float *y);
+
+/* Rewind to t = 0 for a new sequence.  O(1): stale buffer contents are never read
+ * (the first block written onto any position overwrites instead of accumulating). */
+int fi_reset(fi_ctx *ctx);
+
+/* Copy the realised activations a^layer_s for s in [t0, t1) into dst
+ * [t1-t0][B][D]; layer 0 is the input sequence, layer l >= 1 is tanh(y^l).
+ * Requires 0 <= t0 <= t1 <= t (only finalised positions can be read). */
+int fi_read_layer(fi_ctx *ctx, int layer, int t0, int t1, float *dst);
+
+/* Use `stream` (a cudaStream_t, NULL = legacy default stream) for all later work. */
+int fi_set_stream(fi_ctx *ctx, void *stream);
+
+/* Choose the execution path (FI_PATH_WINDOW or FI_PATH_TOKEN). */
+int fi_set_path(fi_ctx *ctx, int path);
+
+/* Enable (1) or disable (0) replay of captured CUDA graphs ([Impl]). */
+int fi_set_graphs(fi_ctx *ctx, int on);
+
+/* Override the tau choice for block size 2^q (FI_TAU_AUTO restores the measured
+ * choice).  FI_EINVAL if the implementation cannot serve that size in this
+ * context (FFT needs the spectrum of that size). */
+int fi_set_tau(fi_ctx *ctx, int q, int impl);
+
+/* Bracket every kernel launch of later runs with CUDA events (on = 1), also inside
+ * captured graphs; off by default.  Toggling re-captures graphs. */
+int fi_set_trace(fi_ctx *ctx, int on);
+
+/* Per kernel class: launches and device time of the most recent run (fi_step,
+ * fi_generate or fi_forward call) made with tracing on.  Synchronises the stream. */
+int fi_trace_read(fi_ctx *ctx, fi_trace *out);
+
+/* Fill *info with the context's shape, state and tau table. */
+int fi_get_info(const fi_ctx *ctx, fi_info *info);
+
+/* The gray block released after the n-th token ([Alg1], 1 <= n <= L-1): its edge
+ * U = lowbit(n), input positions [src_lo, n-1], output positions [n, dst_hi]
+ * (dst_hi clipped to L-1) and the tau implementation the context will use. */
+int fi_debug_schedule(const fi_ctx *ctx, int n, int *U, int *impl, int *src_lo,
+                      int *dst_lo, int *dst_hi);
+
+/* Stand-alone tau ([Lem1]) over `count` independent blocks of edge U, all pointers
+ * DEVICE memory:  out[i][r] (+)= sum_{j<U} blocks[i][j] * taps[i*ldt + U + r - j],
+ * r < U (lags 1 .. 2U-1 of each filter row; ldt >= 2U).  accumulate = 0 overwrites.
+ * impl: FI_TAU_DIRECT (U <= 4096) or FI_TAU_FFT (8 <= U <= 65536, ldt even; all
+ * pointers 8-byte aligned).  Runs on the legacy default stream and
+ * returns after completion.  Used to test each tau kernel in isolation. */
+int fi_tau(int impl, int U, int count, const float *blocks, const float *taps, int ldt,
+           float *out, int accumulate);
+
+/* Message of the last failure on the calling thread ("" if none). */
+const char *fi_last_error(void);
+
+/* Library version string. */
+const char *fi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FI_H_ */

@@ -1,0 +1,197 @@
+"""Python binding of libfi.so, the B200 Flash Inference mixer (see include/fi.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libfi.so.  Arrays may be torch tensors (host or CUDA) or numpy arrays;
+they must be contiguous float32.  If libfi.so has not been built, the first use
+of the library raises ImportError -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+_LIB_PATH = Path(__file__).resolve().parent / "libfi.so"
+
+FI_OK, FI_EINVAL, FI_ECAPACITY, FI_ENOMEM, FI_ECUDA, FI_ESTATE = 0, -1, -2, -3, -4, -5
+FI_TAU_AUTO, FI_TAU_DIRECT, FI_TAU_FFT = 0, 1, 2
+FI_PATH_WINDOW, FI_PATH_TOKEN = 0, 1
+
+
+class FiError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__("fi error %d: %s" % (code, msg))
+        self.code = code
+
+
+class fi_info(ctypes.Structure):
+    _fields_ = [("layers", ctypes.c_int), ("B", ctypes.c_int), ("D", ctypes.c_int), ("L", ctypes.c_int),
+                ("t", ctypes.c_int), ("window", ctypes.c_int), ("chains_per_cta", ctypes.c_int),
+                ("path", ctypes.c_int), ("graphs", ctypes.c_int), ("tau", ctypes.c_int * 32),
+                ("tau_us", (ctypes.c_float * 2) * 32), ("device_bytes", ctypes.c_size_t),
+                ("sm_count", ctypes.c_int), ("launches", ctypes.c_longlong)]
+
+
+FI_K_WINDOW, FI_K_TOKEN_STEP, FI_K_BLOCK_DIRECT, FI_K_BLOCK_FFT, FI_K_BLOCK_SPLIT = range(5)
+FI_K_CLASSES = 5
+KERNEL_CLASS_NAMES = ("window", "token_step", "block_direct", "block_fft", "block_split")
+
+
+class fi_trace(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int * FI_K_CLASSES), ("total_us", ctypes.c_double * FI_K_CLASSES),
+                ("max_us", ctypes.c_double * FI_K_CLASSES)]
+
+
+# Every entry point declared in include/fi.h, with its C signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+SIGNATURES = {
+    "fi_create": (_P, [_I, _I, _I, _I, _P]),
+    "fi_destroy": (None, [_P]),
+    "fi_step": (_I, [_P, _P, _P]),
+    "fi_generate": (_I, [_P, _P, _I, _P]),
+    "fi_forward": (_I, [_P, _P, _I, _P]),
+    "fi_reset": (_I, [_P]),
+    "fi_read_layer": (_I, [_P, _I, _I, _I, _P]),
+    "fi_set_stream": (_I, [_P, _P]),
+    "fi_set_path": (_I, [_P, _I]),
+    "fi_set_graphs": (_I, [_P, _I]),
+    "fi_set_tau": (_I, [_P, _I, _I]),
+    "fi_get_info": (_I, [_P, ctypes.POINTER(fi_info)]),
+    "fi_set_trace": (_I, [_P, _I]),
+    "fi_trace_read": (_I, [_P, ctypes.POINTER(fi_trace)]),
+    "fi_debug_schedule": (_I, [_P, _I] + [ctypes.POINTER(_I)] * 5),
+    "fi_tau": (_I, [_I, _I, _I, _P, _P, _I, _P, _I]),
+    "fi_last_error": (ctypes.c_char_p, []),
+    "fi_version": (ctypes.c_char_p, []),
+}
+
+
+def _load():
+    if not _LIB_PATH.exists():
+        raise ImportError("libfi.so is not built (run __graft_entry__.build() or "
+                          "python -m long_convolution_sequence_b200.build); no fallback exists")
+    lib = ctypes.CDLL(str(_LIB_PATH))
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = None
+
+
+def get_lib():
+    """The loaded libfi.so (raises ImportError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def __getattr__(name):
+    if name == "lib":
+        return get_lib()
+    raise AttributeError(name)
+
+
+def last_error() -> str:
+    return get_lib().fi_last_error().decode()
+
+
+def _check(rc):
+    if rc != FI_OK:
+        raise FiError(rc, last_error())
+
+
+def _ptr(a):
+    """Address of a contiguous float32 torch tensor / numpy array (None -> NULL)."""
+    if a is None:
+        return None
+    if hasattr(a, "data_ptr"):  # torch
+        assert a.is_contiguous(), "tensor must be contiguous"
+        assert str(a.dtype) == "torch.float32", "tensor must be float32"
+        return a.data_ptr()
+    import numpy as np
+    assert isinstance(a, np.ndarray) and a.dtype == np.float32 and a.flags.c_contiguous
+    return a.ctypes.data
+
+
+class FlashInference:
+    """One context (fi_create .. fi_destroy)."""
+
+    def __init__(self, layers: int, B: int, D: int, L: int, filters):
+        self.layers, self.B, self.D, self.L = layers, B, D, L
+        lib = get_lib()
+        h = lib.fi_create(layers, B, D, L, _ptr(filters))
+        if not h:
+            raise FiError(FI_EINVAL, last_error())
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            _lib.fi_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def step(self, x_t, y_t):
+        _check(get_lib().fi_step(self._h, _ptr(x_t), _ptr(y_t)))
+
+    def generate(self, x0, steps: int, out):
+        _check(get_lib().fi_generate(self._h, _ptr(x0), steps, _ptr(out)))
+
+    def forward(self, x, steps: int, y):
+        _check(get_lib().fi_forward(self._h, _ptr(x), steps, _ptr(y)))
+
+    def reset(self):
+        _check(get_lib().fi_reset(self._h))
+
+    def read_layer(self, layer: int, t0: int, t1: int, dst):
+        _check(get_lib().fi_read_layer(self._h, layer, t0, t1, _ptr(dst)))
+
+    def set_stream(self, stream_handle: int):
+        _check(get_lib().fi_set_stream(self._h, stream_handle))
+
+    def set_path(self, path: int):
+        _check(get_lib().fi_set_path(self._h, path))
+
+    def set_graphs(self, on: bool):
+        _check(get_lib().fi_set_graphs(self._h, int(bool(on))))
+
+    def set_tau(self, q: int, impl: int):
+        _check(get_lib().fi_set_tau(self._h, q, impl))
+
+    def set_trace(self, on: bool):
+        _check(get_lib().fi_set_trace(self._h, int(bool(on))))
+
+    def trace(self) -> dict:
+        """{class name: (launches, total_us, max_us)} of the last traced run."""
+        tr = fi_trace()
+        _check(get_lib().fi_trace_read(self._h, ctypes.byref(tr)))
+        return {KERNEL_CLASS_NAMES[k]: (tr.launches[k], tr.total_us[k], tr.max_us[k])
+                for k in range(FI_K_CLASSES) if tr.launches[k]}
+
+    def info(self) -> fi_info:
+        inf = fi_info()
+        _check(get_lib().fi_get_info(self._h, ctypes.byref(inf)))
+        return inf
+
+    def schedule(self, n: int):
+        vals = [ctypes.c_int() for _ in range(5)]
+        _check(get_lib().fi_debug_schedule(self._h, n, *[ctypes.byref(v) for v in vals]))
+        U, impl, src_lo, dst_lo, dst_hi = (v.value for v in vals)
+        return dict(U=U, impl=impl, src_lo=src_lo, dst_lo=dst_lo, dst_hi=dst_hi)
+
+
+def tau(impl: int, U: int, blocks, taps, out, accumulate: bool = False):
+    """Stand-alone tau over independent blocks (device arrays): see fi_tau in fi.h."""
+    count = blocks.shape[0]
+    ldt = taps.shape[1]
+    _check(get_lib().fi_tau(impl, U, count, _ptr(blocks), _ptr(taps), ldt, _ptr(out), int(bool(accumulate))))

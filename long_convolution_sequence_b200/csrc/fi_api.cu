@@ -1,0 +1,989 @@
+// fi_api.cu -- host side of the C-ABI (include/fi.h): context lifetime, the
+// lowbit schedule, the Hybrid tau table, launch sequencing for the window and
+// per-token paths, CUDA-graph capture and replay, host/device staging.
+//
+// Passages followed (web summary of arXiv 2410.12982, "Flash Inference: Near Linear
+// Time Inference for Long Convolution Sequence Models and Beyond"):
+//   section "Kachelung-Strategie (Algorithmus 1)"   -- which block follows which token
+//   section "LCSM-Inferenz-Algorithmus (Algorithmus 2)" -- red cells, blocks, sampler
+//   section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)" -- one launch
+//           carries the blocks of every layer
+//   section "Implementierungsdetails" -- CUDA graphs, FFT precompute, Hybrid tau
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <set>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "fi.h"
+#include "fi_kernels.cuh"
+
+using namespace fi;
+
+namespace {
+
+thread_local char g_err[1024] = "";
+
+int set_err(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+#define CK(call)                                                                               \
+    do {                                                                                       \
+        cudaError_t e_ = (call);                                                               \
+        if (e_ != cudaSuccess)                                                                 \
+            return set_err(e_ == cudaErrorMemoryAllocation ? FI_ENOMEM : FI_ECUDA,             \
+                           "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__,   \
+                           __LINE__);                                                          \
+    } while (0)
+
+constexpr unsigned kMagic = 0xF1C7A5E5u;
+constexpr int kTwLog = 17;          // twiddle table e^{-2 pi i k / 2^17}
+constexpr int kLogSMax = 14;        // largest FFT held by one CTA: 2^14 complex = 128 KB
+constexpr int kFftQMin = 3;         // smallest block size served by FFT (U = 8)
+constexpr int kDirectQMax = 12;     // largest block size served by the direct kernel
+constexpr int kFuseQMax = 4;        // per-token path: blocks up to U = 16 run inside the step kernel
+constexpr int kWinNT = 256;         // threads of the window kernel (1 chain warp + 7 helper warps)
+constexpr int kStepNT = 128;
+constexpr int kDirectNT = 128;
+constexpr size_t kSmemMax = 227 * 1024;
+constexpr int kGraphCache = 8;
+
+struct GraphKey {
+    int path, mode;  // mode: 0 teacher, 1 closed
+    long long t0, steps;
+    const void* x;
+    const void* y;
+    bool operator<(const GraphKey& o) const {
+        return std::tie(path, mode, t0, steps, x, y) < std::tie(o.path, o.mode, o.t0, o.steps, o.x, o.y);
+    }
+};
+
+struct TraceRec {
+    int cls;
+    cudaEvent_t a, b;
+};
+
+struct GraphEntry {
+    cudaGraphExec_t exec = nullptr;
+    std::vector<TraceRec> trace;
+    long long launches = 0;
+};
+
+}  // namespace
+
+struct fi_ctx {
+    unsigned magic = kMagic;
+    int M = 0, B = 0, D = 0, L = 0, P = 0;
+    long long G = 0;
+    int dev = 0, nsm = 0;
+    cudaStream_t stream = nullptr;   // user stream (nullptr = legacy default)
+    cudaStream_t cap = nullptr;      // private stream used to capture graphs
+    float* act = nullptr;            // [(M+1)][G][L]
+    float* h = nullptr;              // [M][D][L]
+    float2* tw = nullptr;            // [2^kTwLog]
+    float2* spec[32] = {};           // per block size 2^q
+    long long spec_stride[32] = {};  // complex entries per (layer, channel)
+    int spec_split[32] = {};         // nsub for split sizes, 1 for single-CTA sizes, 0 none
+    float2* scratch = nullptr;       // split FFT scratch, split_grid CTAs x 4 x (2^14 + 1)
+    int split_grid = 0;
+    int tau[32] = {}, tau_user[32] = {};
+    float tau_us[32][2] = {};
+    int W = 0, kch = 0, win_ncta = 0;
+    size_t win_smem = 0;
+    int path = FI_PATH_WINDOW, graphs = 1;
+    long long t = 0;
+    float* sx = nullptr;  // staging for host inputs
+    size_t sx_n = 0;
+    float* sy = nullptr;  // staging for host outputs
+    size_t sy_n = 0;
+    std::map<GraphKey, GraphEntry> gcache;
+    std::vector<GraphKey> gorder;
+    size_t bytes = 0;
+    // tracing: per-launch event pairs grouped by kernel class
+    int trace_on = 0;
+    std::vector<TraceRec>* rec = nullptr;        // list being filled by enqueue
+    std::vector<TraceRec> eager_trace;           // list of the last eager run
+    const std::vector<TraceRec>* last_trace = nullptr;
+    std::vector<cudaEvent_t> event_pool;
+    size_t event_next = 0;
+    long long launches = 0;                      // kernels launched by runs so far
+    long long enq_launches = 0;                  // kernels enqueued by the current enqueue()
+};
+
+namespace {
+
+bool is_device_ptr(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+int ctz64(long long v) {
+    int q = 0;
+    while (!((v >> q) & 1)) ++q;
+    return q;
+}
+
+// Live contexts: a pointer that was never returned by fi_create, or was destroyed,
+// is rejected without being dereferenced.
+std::mutex g_live_mu;
+std::set<const fi_ctx*> g_live;
+
+int check_ctx(const fi_ctx* c) {
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        if (!c || !g_live.count(c)) return set_err(FI_ESTATE, "null or destroyed context");
+    }
+    if (c->magic != kMagic) return set_err(FI_ESTATE, "null or destroyed context");
+    return FI_OK;
+}
+
+cudaEvent_t pool_event(fi_ctx* c) {
+    if (c->event_next == c->event_pool.size()) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+        c->event_pool.push_back(e);
+    }
+    return c->event_pool[c->event_next++];
+}
+
+// Bracket one launch with events when tracing (also inside graph capture).
+struct LaunchScope {
+    fi_ctx* c;
+    cudaStream_t st;
+    TraceRec r;
+    bool on;
+    LaunchScope(fi_ctx* c_, int cls, cudaStream_t st_) : c(c_), st(st_), on(c_->trace_on && c_->rec) {
+        c->enq_launches++;
+        if (on) {
+            r.cls = cls;
+            r.a = pool_event(c);
+            r.b = pool_event(c);
+            on = r.a && r.b;
+            // external records become event nodes when the stream is being captured
+            if (on) cudaEventRecordWithFlags(r.a, st, cudaEventRecordExternal);
+        }
+    }
+    ~LaunchScope() {
+        if (on) {
+            cudaEventRecordWithFlags(r.b, st, cudaEventRecordExternal);
+            c->rec->push_back(r);
+        }
+    }
+};
+
+template <typename T>
+int dev_alloc(fi_ctx* c, T** p, size_t count) {
+    const char* f = getenv("FI_FAULT");
+    if (f && strstr(f, "alloc")) return set_err(FI_ENOMEM, "injected allocation failure (FI_FAULT=alloc)");
+    cudaError_t e = cudaMalloc((void**)p, count * sizeof(T));
+    if (e != cudaSuccess) {
+        *p = nullptr;
+        cudaGetLastError();
+        return set_err(e == cudaErrorMemoryAllocation ? FI_ENOMEM : FI_ECUDA,
+                       "cudaMalloc(%zu bytes) failed: %s", count * sizeof(T), cudaGetErrorString(e));
+    }
+    c->bytes += count * sizeof(T);
+    return FI_OK;
+}
+
+size_t win_smem_bytes(int W, int M, int B, int kch) {
+    return (size_t)((M + 1) * kch * B + M * kch) * (W + 1) * sizeof(float);
+}
+
+// ---------------------------------------------------------------- kernel launchers
+template <int LOGN>
+int launch_fft_tile_t(const TileArgs& a, cudaStream_t st) {
+    constexpr int NT = (1 << LOGN) / 4 < 32 ? 32 : ((1 << LOGN) / 4 > 1024 ? 1024 : (1 << LOGN) / 4);
+    const size_t smem = sizeof(float2) << LOGN;
+    k_tile_fft<LOGN, NT><<<a.count, NT, smem, st>>>(a);
+    CK(cudaGetLastError());
+    return FI_OK;
+}
+
+int launch_fft_tile(int logn, const TileArgs& a, cudaStream_t st) {
+    switch (logn) {
+        case 3: return launch_fft_tile_t<3>(a, st);
+        case 4: return launch_fft_tile_t<4>(a, st);
+        case 5: return launch_fft_tile_t<5>(a, st);
+        case 6: return launch_fft_tile_t<6>(a, st);
+        case 7: return launch_fft_tile_t<7>(a, st);
+        case 8: return launch_fft_tile_t<8>(a, st);
+        case 9: return launch_fft_tile_t<9>(a, st);
+        case 10: return launch_fft_tile_t<10>(a, st);
+        case 11: return launch_fft_tile_t<11>(a, st);
+        case 12: return launch_fft_tile_t<12>(a, st);
+        case 13: return launch_fft_tile_t<13>(a, st);
+        case 14: return launch_fft_tile_t<14>(a, st);
+        default: return set_err(FI_EINVAL, "no single-CTA FFT for 2^%d points", logn);
+    }
+}
+
+int launch_split_tile(const TileArgs& a, int grid, cudaStream_t st) {
+    constexpr int NT = 1024;
+    const size_t smem = sizeof(float2) << kLogSMax;
+    k_tile_fft_split<kLogSMax, NT><<<grid, NT, smem, st>>>(a);
+    CK(cudaGetLastError());
+    return FI_OK;
+}
+
+int launch_direct_tile(const TileArgs& a, cudaStream_t st) {
+    const size_t smem = (size_t)3 * a.U * sizeof(float);
+    k_tile_direct<kDirectNT, 4><<<a.count, kDirectNT, smem, st>>>(a);
+    CK(cudaGetLastError());
+    return FI_OK;
+}
+
+template <int LOGN>
+int launch_spectra_t(const float* taps, long long ld, int count, int nspec, long long offstep,
+                     float2* spec, const float2* tw, cudaStream_t st) {
+    constexpr int NT = (1 << LOGN) / 4 < 32 ? 32 : ((1 << LOGN) / 4 > 1024 ? 1024 : (1 << LOGN) / 4);
+    const size_t smem = sizeof(float2) << LOGN;
+    // one CTA per (item, offset); chunk the grid to stay below 2^31 CTAs
+    k_spectra<LOGN, NT><<<count * nspec, NT, smem, st>>>(taps, ld, nspec, offstep, spec, tw, kTwLog);
+    CK(cudaGetLastError());
+    return FI_OK;
+}
+
+int launch_spectra(int logn, const float* taps, long long ld, int count, int nspec, long long offstep,
+                   float2* spec, const float2* tw, cudaStream_t st) {
+    switch (logn) {
+        case 3: return launch_spectra_t<3>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 4: return launch_spectra_t<4>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 5: return launch_spectra_t<5>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 6: return launch_spectra_t<6>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 7: return launch_spectra_t<7>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 8: return launch_spectra_t<8>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 9: return launch_spectra_t<9>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 10: return launch_spectra_t<10>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 11: return launch_spectra_t<11>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 12: return launch_spectra_t<12>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 13: return launch_spectra_t<13>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 14: return launch_spectra_t<14>(taps, ld, count, nspec, offstep, spec, tw, st);
+        default: return set_err(FI_EINVAL, "no spectrum kernel for 2^%d points", logn);
+    }
+}
+
+template <int W>
+int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
+    k_window<W, kWinNT><<<c->win_ncta, kWinNT, c->win_smem, st>>>(a);
+    CK(cudaGetLastError());
+    return FI_OK;
+}
+
+int launch_window(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
+    switch (c->W) {
+        case 16: return launch_window_t<16>(c, a, st);
+        case 32: return launch_window_t<32>(c, a, st);
+        case 64: return launch_window_t<64>(c, a, st);
+        case 128: return launch_window_t<128>(c, a, st);
+        case 256: return launch_window_t<256>(c, a, st);
+        default: return set_err(FI_EINVAL, "unsupported window %d", c->W);
+    }
+}
+
+// Dynamic shared memory above 48 KB must be enabled per kernel before the first
+// launch (and before any graph capture); done once per process.
+template <int LOGN>
+int attr_fft() {
+    constexpr int NT = (1 << LOGN) / 4 < 32 ? 32 : ((1 << LOGN) / 4 > 1024 ? 1024 : (1 << LOGN) / 4);
+    const int smem = (int)(sizeof(float2) << LOGN);
+    CK(cudaFuncSetAttribute(k_tile_fft<LOGN, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    CK(cudaFuncSetAttribute(k_spectra<LOGN, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    return FI_OK;
+}
+
+int set_all_attrs() {
+    static int done = 0;
+    if (done) return FI_OK;
+    int rc = 0;
+    rc |= attr_fft<3>() | attr_fft<4>() | attr_fft<5>() | attr_fft<6>() | attr_fft<7>() | attr_fft<8>();
+    rc |= attr_fft<9>() | attr_fft<10>() | attr_fft<11>() | attr_fft<12>() | attr_fft<13>() | attr_fft<14>();
+    if (rc) return FI_ECUDA;
+    CK(cudaFuncSetAttribute(k_tile_fft_split<kLogSMax, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)(sizeof(float2) << kLogSMax)));
+    CK(cudaFuncSetAttribute(k_tile_direct<kDirectNT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)(3 * (1 << kDirectQMax) * sizeof(float))));
+    CK(cudaFuncSetAttribute(k_window<16, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<32, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<64, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<128, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<256, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    done = 1;
+    return FI_OK;
+}
+
+TileArgs stack_tile_args(const fi_ctx* c, long long n) {
+    TileArgs a;
+    memset(&a, 0, sizeof(a));
+    a.act = c->act;
+    a.h = c->h;
+    a.L = c->L;
+    a.G = c->G;
+    a.D = c->D;
+    a.n = n;
+    a.U = (int)lowbit(n);
+    a.count = (int)(c->M * c->G);
+    a.overwrite = is_pow2(n) ? 1 : 0;
+    a.tw = c->tw;
+    a.twlog = kTwLog;
+    return a;
+}
+
+// The gray blocks of every layer released after the n-th token, one launch
+// (section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)").
+int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st) {
+    TileArgs a = stack_tile_args(c, n);
+    const int q = ctz64(n);
+    const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
+                    : (c->spec_split[q] > 1 ? FI_K_BLOCK_SPLIT : FI_K_BLOCK_FFT);
+    LaunchScope scope(c, cls, st);
+    if (impl == FI_TAU_DIRECT) return launch_direct_tile(a, st);
+    a.spec = c->spec[q];
+    a.spec_stride = c->spec_stride[q];
+    if (c->spec_split[q] > 1) {
+        a.nsub = c->spec_split[q];
+        a.scratch = c->scratch;
+        return launch_split_tile(a, c->split_grid, st);
+    }
+    return launch_fft_tile(q, a, st);
+}
+
+int upload_twiddles(fi_ctx* c) {
+    const int nt = 1 << kTwLog;
+    std::vector<float2> tw(nt);
+    for (int k = 0; k < nt; ++k) {
+        double ang = -2.0 * M_PI * (double)k / (double)nt;
+        tw[k] = make_float2((float)cos(ang), (float)sin(ang));
+    }
+    int rc = dev_alloc(c, &c->tw, (size_t)nt);
+    if (rc) return rc;
+    CK(cudaMemcpy(c->tw, tw.data(), sizeof(float2) * nt, cudaMemcpyHostToDevice));
+    return FI_OK;
+}
+
+int tau_impl(fi_ctx* tmp, int impl, int U, int q, int count, const float* blocks, const float* taps, int ldt,
+             float* out, int accumulate) {
+    TileArgs a;
+    memset(&a, 0, sizeof(a));
+    a.flat = 1;
+    a.fin = blocks;
+    a.fout = out;
+    a.ftaps = taps;
+    a.ldt = ldt;
+    a.U = U;
+    a.count = count;
+    a.overwrite = accumulate ? 0 : 1;
+    cudaStream_t st = nullptr;
+    int rc;
+    if (impl == FI_TAU_DIRECT) {
+        rc = launch_direct_tile(a, st);
+    } else {
+        if ((rc = upload_twiddles(tmp))) return rc;
+        a.tw = tmp->tw;
+        a.twlog = kTwLog;
+        if (q <= kLogSMax) {
+            if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * (U + 1)))) return rc;
+            if ((rc = launch_spectra(q, taps, ldt, count, 1, 0, tmp->spec[0], tmp->tw, st))) return rc;
+            a.spec = tmp->spec[0];
+            a.spec_stride = U + 1;
+            rc = launch_fft_tile(q, a, st);
+        } else {
+            const long long S = 1LL << kLogSMax;
+            const int nsub = (int)(U / S), nspec = 2 * nsub - 1;
+            int nsm = 0, dev = 0;
+            CK(cudaGetDevice(&dev));
+            CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+            if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * nspec * (S + 1)))) return rc;
+            if ((rc = launch_spectra(kLogSMax, taps, ldt, count, nspec, S, tmp->spec[0], tmp->tw, st))) return rc;
+            if ((rc = dev_alloc(tmp, &tmp->scratch, (size_t)nsm * nsub * (S + 1)))) return rc;
+            a.spec = tmp->spec[0];
+            a.spec_stride = (long long)nspec * (S + 1);
+            a.nsub = nsub;
+            a.scratch = tmp->scratch;
+            rc = launch_split_tile(a, nsm, st);
+        }
+    }
+    if (rc) return rc;
+    CK(cudaStreamSynchronize(st));
+    return FI_OK;
+}
+
+int tau_of(const fi_ctx* c, int q) { return c->tau_user[q] ? c->tau_user[q] : c->tau[q]; }
+
+// ---------------------------------------------------------------- launch sequences
+int enqueue_token(fi_ctx* c, long long t, const float* x, float* y, int closed, cudaStream_t st) {
+    StepArgs a;
+    a.act = c->act;
+    a.h = c->h;
+    a.M = c->M;
+    a.D = c->D;
+    a.L = c->L;
+    a.G = c->G;
+    a.t = t;
+    a.x = x;
+    a.y = y;
+    a.closed = closed;
+    a.fuseU = 0;
+    const long long n = t + 1;
+    int q = -1, impl = 0;
+    if (n < c->L) {
+        q = ctz64(n);
+        impl = tau_of(c, q);
+        if (q <= kFuseQMax && impl == FI_TAU_DIRECT) a.fuseU = 1 << q;
+    }
+    const int grid = (int)((c->G + 31) / 32);
+    {
+        LaunchScope scope(c, FI_K_TOKEN_STEP, st);
+        k_token_step<kStepNT><<<grid, kStepNT, 0, st>>>(a);
+        CK(cudaGetLastError());
+    }
+    if (n < c->L && a.fuseU == 0) return launch_block(c, n, impl, st);
+    return FI_OK;
+}
+
+int enqueue_window_path(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed,
+                        cudaStream_t st) {
+    const long long W = c->W, L = c->L, end = t0 + steps;
+    long long t = t0;
+    while (t < end) {
+        const long long k = t / W;
+        const long long wend = std::min((k + 1) * W, L);
+        const long long t1 = std::min(end, wend);
+        WinArgs a;
+        a.act = c->act;
+        a.h = c->h;
+        a.M = c->M;
+        a.B = c->B;
+        a.D = c->D;
+        a.L = L;
+        a.G = c->G;
+        a.t0 = t;
+        a.t1 = t1;
+        a.tx = t0;
+        a.x = closed ? (t == t0 ? x : nullptr) : x;
+        a.out = out;
+        a.closed = closed;
+        a.kch = c->kch;
+        int rc;
+        {
+            LaunchScope scope(c, FI_K_WINDOW, st);
+            rc = launch_window(c, a, st);
+        }
+        if (rc) return rc;
+        if (t1 == (k + 1) * W && t1 < L) {
+            rc = launch_block(c, t1, tau_of(c, ctz64(t1)), st);
+            if (rc) return rc;
+        }
+        t = t1;
+    }
+    return FI_OK;
+}
+
+int enqueue(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed, cudaStream_t st) {
+    if (c->path == FI_PATH_WINDOW && c->W > 0) return enqueue_window_path(c, t0, steps, x, out, closed, st);
+    for (long long k = 0; k < steps; ++k) {
+        const float* xk = closed ? (k == 0 ? x : nullptr) : x + k * c->G;
+        int rc = enqueue_token(c, t0 + k, xk, out + k * c->G, closed, st);
+        if (rc) return rc;
+    }
+    return FI_OK;
+}
+
+void drop_graphs(fi_ctx* c) {
+    if (c->last_trace != &c->eager_trace) c->last_trace = nullptr;
+    for (auto& kv : c->gcache) cudaGraphExecDestroy(kv.second.exec);
+    c->gcache.clear();
+    c->gorder.clear();
+}
+
+// Run a launch sequence, from a captured graph when enabled (section
+// "Implementierungsdetails": CUDA graphs remove the per-launch CPU overhead).
+int run(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed) {
+    const bool window = c->path == FI_PATH_WINDOW && c->W > 0;
+    c->enq_launches = 0;
+    if (!c->graphs || !window) {
+        c->eager_trace.clear();
+        c->event_next = 0;
+        c->rec = &c->eager_trace;
+        int rc = enqueue(c, t0, steps, x, out, closed, c->stream);
+        c->rec = nullptr;
+        c->last_trace = &c->eager_trace;
+        c->launches += c->enq_launches;
+        return rc;
+    }
+    GraphKey key{c->path, closed, t0, steps, x, out};
+    auto it = c->gcache.find(key);
+    if (it == c->gcache.end()) {
+        if ((int)c->gorder.size() >= kGraphCache) {
+            GraphKey old = c->gorder.front();
+            c->gorder.erase(c->gorder.begin());
+            if (c->last_trace == &c->gcache[old].trace) c->last_trace = nullptr;
+            cudaGraphExecDestroy(c->gcache[old].exec);
+            c->gcache.erase(old);
+        }
+        GraphEntry ent;
+        CK(cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed));
+        c->rec = &ent.trace;
+        int rc = enqueue(c, t0, steps, x, out, closed, c->cap);
+        c->rec = nullptr;
+        cudaGraph_t graph = nullptr;
+        cudaError_t e = cudaStreamEndCapture(c->cap, &graph);
+        if (rc) {
+            if (graph) cudaGraphDestroy(graph);
+            return rc;
+        }
+        if (e != cudaSuccess) return set_err(FI_ECUDA, "graph capture failed: %s", cudaGetErrorString(e));
+        const char* f = getenv("FI_FAULT");
+        if (f && strstr(f, "capture")) {
+            cudaGraphDestroy(graph);
+            return set_err(FI_ECUDA, "injected graph capture failure (FI_FAULT=capture)");
+        }
+        e = cudaGraphInstantiate(&ent.exec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) return set_err(FI_ECUDA, "graph instantiate failed: %s", cudaGetErrorString(e));
+        ent.launches = c->enq_launches;
+        it = c->gcache.emplace(key, std::move(ent)).first;
+        c->gorder.push_back(key);
+    }
+    CK(cudaGraphLaunch(it->second.exec, c->stream));
+    c->last_trace = &it->second.trace;
+    c->launches += it->second.launches;
+    return FI_OK;
+}
+
+int ensure_stage(fi_ctx* c, float** buf, size_t* cap, size_t n) {
+    if (*cap >= n) return FI_OK;
+    if (*buf) {
+        CK(cudaStreamSynchronize(c->stream));
+        cudaFree(*buf);
+        c->bytes -= *cap * sizeof(float);
+        *buf = nullptr;
+        *cap = 0;
+        drop_graphs(c);  // graphs may reference the old staging buffer
+    }
+    int rc = dev_alloc(c, buf, n);
+    if (rc) return rc;
+    *cap = n;
+    return FI_OK;
+}
+
+// ---------------------------------------------------------------- setup
+int choose_window(fi_ctx* c) {
+    const char* env = getenv("FI_WINDOW");
+    int forced = env ? atoi(env) : 0;
+    if (c->B > 32) return FI_OK;  // chain lanes: one warp per CTA
+    int kch = (int)((c->D + c->nsm - 1) / c->nsm);
+    if (kch * c->B > 32) kch = std::max(1, 32 / c->B);
+    const int ncta = (c->D + kch - 1) / kch;
+    const int per_sm = (ncta + c->nsm - 1) / c->nsm;
+    const int cand[] = {256, 128, 64, 32, 16};
+    for (int W : cand) {
+        if (forced && W != forced) continue;
+        if (W > c->L) continue;
+        size_t sm = win_smem_bytes(W, c->M, c->B, kch);
+        if (sm > kSmemMax || sm * per_sm > 228 * 1024) continue;
+        c->W = W;
+        c->kch = kch;
+        c->win_ncta = ncta;
+        c->win_smem = sm;
+        return FI_OK;
+    }
+    return FI_OK;  // W = 0: window path unavailable, per-token path only
+}
+
+float time_launch(fi_ctx* c, long long n, int impl, int reps) {
+    cudaEvent_t e0, e1;
+    cudaEventCreate(&e0);
+    cudaEventCreate(&e1);
+    if (launch_block(c, n, impl, c->cap)) return -1.f;
+    cudaEventRecord(e0, c->cap);
+    for (int r = 0; r < reps; ++r)
+        if (launch_block(c, n, impl, c->cap)) return -1.f;
+    cudaEventRecord(e1, c->cap);
+    cudaEventSynchronize(e1);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, e0, e1);
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    return ms * 1000.f / reps;
+}
+
+// Hybrid tau: time each implementation able to serve block size 2^q and keep the
+// faster (ties go to direct).  The timing launches write into positions that the
+// first real block onto them overwrites, so they leave no trace.
+int autotune(fi_ctx* c) {
+    const char* env = getenv("FI_TAU");  // "q:impl,q:impl" with impl d|f
+    for (int q = 0; q < c->P; ++q) {
+        const long long U = 1LL << q;
+        const bool can_d = q <= kDirectQMax;
+        const bool can_f = c->spec[q] != nullptr;
+        float td = 0.f, tf = 0.f;
+        if (can_d && can_f) {
+            td = time_launch(c, U, FI_TAU_DIRECT, 3);
+            tf = time_launch(c, U, FI_TAU_FFT, 3);
+            if (td < 0 || tf < 0) return FI_ECUDA;
+        }
+        c->tau_us[q][0] = td;
+        c->tau_us[q][1] = tf;
+        if (can_d && can_f) c->tau[q] = (tf < td) ? FI_TAU_FFT : FI_TAU_DIRECT;
+        else c->tau[q] = can_f ? FI_TAU_FFT : FI_TAU_DIRECT;
+        (void)U;
+    }
+    if (env) {
+        const char* p = env;
+        while (*p) {
+            int q = atoi(p);
+            const char* colon = strchr(p, ':');
+            if (!colon) break;
+            char k = colon[1];
+            if (q >= 0 && q < c->P) {
+                if (k == 'd' && q <= kDirectQMax) c->tau[q] = FI_TAU_DIRECT;
+                if (k == 'f' && c->spec[q]) c->tau[q] = FI_TAU_FFT;
+            }
+            const char* comma = strchr(colon, ',');
+            if (!comma) break;
+            p = comma + 1;
+        }
+    }
+    return FI_OK;
+}
+
+void free_ctx(fi_ctx* c) {
+    if (!c) return;
+    cudaStreamSynchronize(c->stream);
+    drop_graphs(c);
+    cudaFree(c->act);
+    cudaFree(c->h);
+    cudaFree(c->tw);
+    for (int q = 0; q < 32; ++q) cudaFree(c->spec[q]);
+    cudaFree(c->scratch);
+    cudaFree(c->sx);
+    cudaFree(c->sy);
+    for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
+    if (c->cap) cudaStreamDestroy(c->cap);
+    c->magic = 0;
+    delete c;
+}
+
+int create_impl(fi_ctx* c, const float* filters) {
+    int rc0 = set_all_attrs();
+    if (rc0) return rc0;
+    CK(cudaGetDevice(&c->dev));
+    CK(cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev));
+    CK(cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking));
+    const long long M = c->M, D = c->D, L = c->L, G = c->G;
+    int rc;
+    if ((rc = dev_alloc(c, &c->act, (size_t)(M + 1) * G * L))) return rc;
+    if ((rc = dev_alloc(c, &c->h, (size_t)M * D * L))) return rc;
+    CK(cudaMemcpyAsync(c->h, filters, sizeof(float) * M * D * L, cudaMemcpyDefault, c->cap));
+    // twiddles from fp64 host trigonometry
+    if ((rc = upload_twiddles(c))) return rc;
+    // filter spectra for every FFT-served block size
+    for (int q = kFftQMin; q < c->P; ++q) {
+        const long long U = 1LL << q;
+        if (q <= kLogSMax) {
+            c->spec_split[q] = 1;
+            c->spec_stride[q] = U + 1;
+            if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * (U + 1)))) return rc;
+            if ((rc = launch_spectra(q, c->h, L, (int)(M * D), 1, 0, c->spec[q], c->tw, c->cap))) return rc;
+        } else {
+            const long long S = 1LL << kLogSMax;
+            const int nsub = (int)(U / S);
+            const int nspec = 2 * nsub - 1;
+            c->spec_split[q] = nsub;
+            c->spec_stride[q] = (long long)nspec * (S + 1);
+            if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * nspec * (S + 1)))) return rc;
+            if ((rc = launch_spectra(kLogSMax, c->h, L, (int)(M * D), nspec, S, c->spec[q], c->tw, c->cap)))
+                return rc;
+        }
+    }
+    if (c->P - 1 > kLogSMax) {
+        c->split_grid = c->nsm;
+        const long long S = 1LL << kLogSMax;
+        const int nsub_max = (int)((1LL << (c->P - 1)) / S);
+        if ((rc = dev_alloc(c, &c->scratch, (size_t)c->split_grid * nsub_max * (S + 1)))) return rc;
+    }
+    CK(cudaStreamSynchronize(c->cap));
+    if ((rc = choose_window(c))) return rc;
+    if ((rc = autotune(c))) return rc;
+    CK(cudaStreamSynchronize(c->cap));
+    return FI_OK;
+}
+
+
+}  // namespace
+
+// ====================================================================== C-ABI
+extern "C" {
+
+const char* fi_last_error(void) { return g_err; }
+
+const char* fi_version(void) { return "fi-b200 0.1 (sm_100a)"; }
+
+fi_ctx* fi_create(int layers, int B, int D, int L, const float* filters) {
+    g_err[0] = 0;
+    if (layers < 1 || B < 1 || D < 1 || L < 2 || (L & (L - 1)) || !filters) {
+        set_err(FI_EINVAL, "fi_create: need layers, B, D >= 1, L a power of two >= 2, filters != NULL "
+                           "(got %d, %d, %d, %d, %p)", layers, B, D, L, (const void*)filters);
+        return nullptr;
+    }
+    const long long G = (long long)B * D;
+    if ((long long)(layers + 1) * G * L > (1LL << 40)) {
+        set_err(FI_EINVAL, "fi_create: buffers too large");
+        return nullptr;
+    }
+    fi_ctx* c = new fi_ctx();
+    c->M = layers;
+    c->B = B;
+    c->D = D;
+    c->L = L;
+    c->G = G;
+    while ((1 << c->P) < L) ++c->P;
+    int rc = create_impl(c, filters);
+    if (rc) {
+        std::string msg = g_err;
+        free_ctx(c);
+        cudaGetLastError();
+        set_err(rc, "%s", msg.c_str());
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    g_live.insert(c);
+    return c;
+}
+
+void fi_destroy(fi_ctx* ctx) {
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        if (!ctx || !g_live.count(ctx)) return;
+        g_live.erase(ctx);
+    }
+    free_ctx(ctx);
+}
+
+int fi_reset(fi_ctx* ctx) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    ctx->t = 0;
+    return FI_OK;
+}
+
+static int run_call(fi_ctx* c, const float* x, int steps, float* out, int closed) {
+    int rc = check_ctx(c);
+    if (rc) return rc;
+    if (steps < 0) return set_err(FI_EINVAL, "steps must be >= 0");
+    if (c->t + steps > c->L)
+        return set_err(FI_ECAPACITY, "t=%lld + steps=%d exceeds capacity L=%d", c->t, steps, c->L);
+    if (steps == 0) return FI_OK;
+    if (!out) return set_err(FI_EINVAL, "output pointer is NULL");
+    if (!closed && !x) return set_err(FI_EINVAL, "input pointer is NULL");
+    if (closed && !x && c->t == 0) return set_err(FI_EINVAL, "closed loop at t=0 needs x0");
+    const long long G = c->G;
+    const float* xd = x;
+    float* od = out;
+    const bool x_host = x && !is_device_ptr(x);
+    const bool o_host = !is_device_ptr(out);
+    if (x_host) {
+        const size_t nx = closed ? (size_t)G : (size_t)G * steps;
+        if ((rc = ensure_stage(c, &c->sx, &c->sx_n, nx))) return rc;
+        CK(cudaMemcpyAsync(c->sx, x, nx * sizeof(float), cudaMemcpyHostToDevice, c->stream));
+        xd = c->sx;
+    }
+    if (o_host) {
+        if ((rc = ensure_stage(c, &c->sy, &c->sy_n, (size_t)G * steps))) return rc;
+        od = c->sy;
+    }
+    rc = run(c, c->t, steps, xd, od, closed);
+    if (rc) return rc;
+    c->t += steps;
+    if (o_host) {
+        CK(cudaMemcpyAsync(out, od, sizeof(float) * G * steps, cudaMemcpyDeviceToHost, c->stream));
+        CK(cudaStreamSynchronize(c->stream));
+    }
+    return FI_OK;
+}
+
+int fi_step(fi_ctx* ctx, const float* x_t, float* y_t) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (!x_t || !y_t) return set_err(FI_EINVAL, "fi_step: x_t and y_t must be non-NULL");
+    // one token: the per-token sequence is the natural form
+    const int saved = ctx->path;
+    ctx->path = FI_PATH_TOKEN;
+    rc = run_call(ctx, x_t, 1, y_t, 0);
+    ctx->path = saved;
+    return rc;
+}
+
+int fi_generate(fi_ctx* ctx, const float* x0, int steps, float* out) { return run_call(ctx, x0, steps, out, 1); }
+
+int fi_forward(fi_ctx* ctx, const float* x, int steps, float* y) { return run_call(ctx, x, steps, y, 0); }
+
+int fi_read_layer(fi_ctx* ctx, int layer, int t0, int t1, float* dst) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (layer < 0 || layer > ctx->M || t0 < 0 || t1 < t0 || t1 > ctx->t || !dst)
+        return set_err(FI_EINVAL, "fi_read_layer: need 0 <= layer <= %d, 0 <= t0 <= t1 <= t=%lld", ctx->M,
+                       ctx->t);
+    if (t1 == t0) return FI_OK;
+    const size_t n = (size_t)(t1 - t0) * ctx->G;
+    const bool host = !is_device_ptr(dst);
+    float* d = dst;
+    if (host) {
+        if ((rc = ensure_stage(ctx, &ctx->sy, &ctx->sy_n, n))) return rc;
+        d = ctx->sy;
+    }
+    const int grid = (int)std::min<size_t>((n + 255) / 256, 65535);
+    k_read_layer<<<grid, 256, 0, ctx->stream>>>(ctx->act, ctx->L, ctx->G, layer, t0, t1, d);
+    CK(cudaGetLastError());
+    if (host) {
+        CK(cudaMemcpyAsync(dst, d, n * sizeof(float), cudaMemcpyDeviceToHost, ctx->stream));
+        CK(cudaStreamSynchronize(ctx->stream));
+    }
+    return FI_OK;
+}
+
+int fi_set_stream(fi_ctx* ctx, void* stream) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    ctx->stream = (cudaStream_t)stream;
+    return FI_OK;
+}
+
+int fi_set_path(fi_ctx* ctx, int path) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (path != FI_PATH_WINDOW && path != FI_PATH_TOKEN) return set_err(FI_EINVAL, "unknown path %d", path);
+    if (path == FI_PATH_WINDOW && ctx->W == 0)
+        return set_err(FI_EINVAL, "window path unavailable for this shape (shared memory)");
+    ctx->path = path;
+    return FI_OK;
+}
+
+int fi_set_graphs(fi_ctx* ctx, int on) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    ctx->graphs = on ? 1 : 0;
+    return FI_OK;
+}
+
+int fi_set_tau(fi_ctx* ctx, int q, int impl) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (q < 0 || q >= ctx->P) return set_err(FI_EINVAL, "block size 2^%d out of range", q);
+    if (impl == FI_TAU_DIRECT && q > kDirectQMax)
+        return set_err(FI_EINVAL, "direct tau limited to U <= %d", 1 << kDirectQMax);
+    if (impl == FI_TAU_FFT && !ctx->spec[q]) return set_err(FI_EINVAL, "no spectrum for U = %d", 1 << q);
+    if (impl != FI_TAU_AUTO && impl != FI_TAU_DIRECT && impl != FI_TAU_FFT)
+        return set_err(FI_EINVAL, "unknown tau implementation %d", impl);
+    ctx->tau_user[q] = impl;
+    drop_graphs(ctx);
+    return FI_OK;
+}
+
+int fi_get_info(const fi_ctx* ctx, fi_info* info) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (!info) return set_err(FI_EINVAL, "info is NULL");
+    memset(info, 0, sizeof(*info));
+    info->layers = ctx->M;
+    info->B = ctx->B;
+    info->D = ctx->D;
+    info->L = ctx->L;
+    info->t = (int)ctx->t;
+    info->window = ctx->W;
+    info->chains_per_cta = ctx->kch * ctx->B;
+    info->path = (ctx->path == FI_PATH_WINDOW && ctx->W) ? FI_PATH_WINDOW : FI_PATH_TOKEN;
+    info->graphs = ctx->graphs;
+    for (int q = 0; q < ctx->P && q < 32; ++q) {
+        info->tau[q] = tau_of(ctx, q);
+        info->tau_us[q][0] = ctx->tau_us[q][0];
+        info->tau_us[q][1] = ctx->tau_us[q][1];
+    }
+    info->device_bytes = ctx->bytes;
+    info->sm_count = ctx->nsm;
+    info->launches = ctx->launches;
+    return FI_OK;
+}
+
+int fi_set_trace(fi_ctx* ctx, int on) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if ((on ? 1 : 0) != ctx->trace_on) drop_graphs(ctx);  // recapture with or without events
+    ctx->trace_on = on ? 1 : 0;
+    return FI_OK;
+}
+
+int fi_trace_read(fi_ctx* ctx, fi_trace* out) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (!out) return set_err(FI_EINVAL, "fi_trace_read: out is NULL");
+    memset(out, 0, sizeof(*out));
+    if (!ctx->last_trace) return FI_OK;
+    CK(cudaStreamSynchronize(ctx->stream));
+    for (const TraceRec& r : *ctx->last_trace) {
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, r.a, r.b));
+        if (r.cls < 0 || r.cls >= FI_K_CLASSES) continue;
+        out->launches[r.cls] += 1;
+        out->total_us[r.cls] += 1000.0 * ms;
+        if (1000.0 * ms > out->max_us[r.cls]) out->max_us[r.cls] = 1000.0 * ms;
+    }
+    return FI_OK;
+}
+
+int fi_debug_schedule(const fi_ctx* ctx, int n, int* U, int* impl, int* src_lo, int* dst_lo, int* dst_hi) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (n < 1 || n > ctx->L - 1) return set_err(FI_EINVAL, "n must be in [1, L-1]");
+    const long long u = lowbit(n);
+    if (U) *U = (int)u;
+    if (impl) *impl = tau_of(ctx, ctz64(n));
+    if (src_lo) *src_lo = (int)(n - u);
+    if (dst_lo) *dst_lo = n;
+    if (dst_hi) *dst_hi = (int)std::min<long long>(n + u - 1, ctx->L - 1);
+    return FI_OK;
+}
+
+int fi_tau(int impl, int U, int count, const float* blocks, const float* taps, int ldt, float* out,
+           int accumulate) {
+    if (U < 1 || (U & (U - 1)) || count < 1 || !blocks || !taps || !out || ldt < 2 * U)
+        return set_err(FI_EINVAL, "fi_tau: need U a power of two, count >= 1, ldt >= 2U, non-NULL pointers");
+    const int q = ctz64(U);
+    if (impl != FI_TAU_DIRECT && impl != FI_TAU_FFT) return set_err(FI_EINVAL, "fi_tau: unknown impl %d", impl);
+    if (impl == FI_TAU_DIRECT && q > kDirectQMax)
+        return set_err(FI_EINVAL, "fi_tau: direct tau limited to U <= %d", 1 << kDirectQMax);
+    if (impl == FI_TAU_FFT && (ldt & 1))
+        return set_err(FI_EINVAL, "fi_tau: FFT tau reads taps in pairs; ldt must be even");
+    if (impl == FI_TAU_FFT && (q < kFftQMin || q > kLogSMax + 2))
+        return set_err(FI_EINVAL, "fi_tau: FFT tau needs %d <= U <= %d", 1 << kFftQMin, 1 << (kLogSMax + 2));
+    int rc = set_all_attrs();
+    if (rc) return rc;
+    fi_ctx tmp;  // holds this call's temporary allocations
+    rc = tau_impl(&tmp, impl, U, q, count, blocks, taps, ldt, out, accumulate);
+    cudaFree(tmp.tw);
+    cudaFree(tmp.spec[0]);
+    cudaFree(tmp.scratch);
+    tmp.magic = 0;
+    return rc;
+}
+
+}  // extern "C"

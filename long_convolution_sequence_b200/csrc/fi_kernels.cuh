@@ -1,0 +1,710 @@
+// fi_kernels.cuh -- device code of the B200 Flash Inference mixer (sm_100a).
+//
+// Notation (web summary of arXiv 2410.12982, "Flash Inference: Near Linear Time
+// Inference for Long Convolution Sequence Models and Beyond"):
+//   * section "LCSM-spezifische Definition": y^l_t = sum_{s<=t} h^l[c][t-s] a^{l-1}_s
+//   * section "Kachelung-Strategie (Algorithmus 1)": after the n-th token (n = t+1)
+//     the gray block of edge U = lowbit(n) adds tau of inputs [n-U, n-1] onto
+//     outputs [n, n+U-1]; the red cell adds h_0 a_t onto y_t.
+//   * section "LCSM-Inferenz-Algorithmus (Algorithmus 2)": layers in order,
+//     block = tanh, sampler = tanh.
+//   * section "Speicheroptimierung": one buffer per layer; position s holds the
+//     running sum b^l_s until token s is processed, then a^l_s.
+//   * section "Zirkulaere Faltungs-Trick": a block is a 2U-point circular
+//     convolution whose outputs [U, 2U-1] are free of wrap-around.
+//
+// Storage ("act"): [(M+1)][G][L] fp32, G = B*D chains (g = b*D + c), layer 0 holds
+// the input sequence.  Filters ("h"): [M][D][L] fp32.  Spectra: per block size,
+// [M][D][nspec][N+1] complex64.
+//
+// First-writer rule: the block released after token n = 2^p is the first one to
+// touch positions [2^p, 2^(p+1)-1]; it stores with "=" and every later block
+// accumulates.  Position 0 is never written by a block; its running sum is 0.
+// Hence no buffer ever needs clearing, and rewinding a context is O(1).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fi {
+
+// ----------------------------------------------------------------- utilities
+__host__ __device__ __forceinline__ long long lowbit(long long n) { return n & (-n); }
+__host__ __device__ __forceinline__ bool is_pow2(long long n) { return n > 0 && (n & (n - 1)) == 0; }
+
+// tanh(y) = 1 - 2 / (1 + 2^(2 y log2(e))), from the definition of tanh through the
+// exponential, evaluated with the SFU's base-2 exponential and reciprocal.  Absolute
+// error below 3e-7 over the reals (checked against fp64 tanh and CUDA's tanhf by
+// the GPU tests); saturates exactly to +-1 for large |y|.
+__device__ __forceinline__ float sfu_ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float sfu_rcp(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float act_tanh(float y) {
+#ifdef FI_TANH_LIBM
+    return tanhf(y);
+#else
+    const float two_log2e = 2.8853900817779268f;  // 2 / ln 2
+    float e = sfu_ex2(two_log2e * y);
+    float r = sfu_rcp(1.0f + e);
+    return fmaf(-2.0f, r, 1.0f);
+#endif
+}
+
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+    return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float2 conjf2(float2 a) { return make_float2(a.x, -a.y); }
+
+// ----------------------------------------------------------------- tile addressing
+// A "tile" is one gray block for one (layer, chain), or one stand-alone tau item.
+struct TileArgs {
+    // stack addressing
+    float* act;
+    const float* h;
+    long long L;
+    long long G;
+    int D;
+    long long n;  // block released after the n-th token
+    // flat addressing (stand-alone tau): in + i*U, out + i*U, taps + i*ldt
+    const float* fin;
+    float* fout;
+    const float* ftaps;
+    long long ldt;
+    int flat;
+    // common
+    int U;
+    int count;       // number of tiles
+    int overwrite;   // 1: store, 0: accumulate
+    const float2* spec;  // spectra of this block size (FFT)
+    long long spec_stride;  // complex entries per item
+    const float2* tw;    // e^{-2 pi i k / 2^twlog}, k < 2^twlog
+    int twlog;
+    float2* scratch;     // split FFT: per-CTA spectra of the input sub-blocks
+    int nsub;            // split FFT: U / S
+};
+
+struct TilePtrs {
+    const float* in;
+    float* out;
+    const float* taps;
+    const float2* spec;
+};
+
+__device__ __forceinline__ TilePtrs tile_ptrs(const TileArgs& a, long long item) {
+    TilePtrs p;
+    if (a.flat) {
+        p.in = a.fin + item * a.U;
+        p.out = a.fout + item * a.U;
+        p.taps = a.ftaps + item * a.ldt;
+        p.spec = a.spec ? a.spec + item * a.spec_stride : nullptr;
+    } else {
+        long long l1 = item / a.G;  // layer - 1
+        long long g = item - l1 * a.G;
+        long long c = g % a.D;
+        p.in = a.act + (l1 * a.G + g) * a.L + (a.n - a.U);
+        p.out = a.act + ((l1 + 1) * a.G + g) * a.L + a.n;
+        p.taps = a.h + (l1 * a.D + c) * a.L;
+        p.spec = a.spec ? a.spec + (l1 * a.D + c) * a.spec_stride : nullptr;
+    }
+    return p;
+}
+
+// ----------------------------------------------------------------- direct tau
+// out[r] (+)= sum_{j<U} in[j] * taps[U + r - j], one tile per CTA, operands staged
+// in shared memory (block U floats, taps 2U floats).
+template <int NT, int RG>
+__global__ void __launch_bounds__(NT) k_tile_direct(TileArgs a) {
+    extern __shared__ float sm[];
+    const int U = a.U;
+    float* sin = sm;
+    float* stap = sm + U;
+    TilePtrs p = tile_ptrs(a, blockIdx.x);
+    for (int j = threadIdx.x; j < U; j += NT) sin[j] = p.in[j];
+    for (int k = threadIdx.x; k < 2 * U; k += NT) stap[k] = p.taps[k];
+    __syncthreads();
+    // each thread owns RG consecutive rows of a strided group
+    const int ngrp = (U + RG - 1) / RG;
+    for (int grp = threadIdx.x; grp < ngrp; grp += NT) {
+        const int r0 = grp * RG;
+        float acc[RG];
+#pragma unroll
+        for (int q = 0; q < RG; ++q) acc[q] = 0.f;
+        for (int j = 0; j < U; ++j) {
+            const float x = sin[j];
+#pragma unroll
+            for (int q = 0; q < RG; ++q) {
+                int lag = U + r0 + q - j;
+                if (r0 + q < U) acc[q] = fmaf(x, stap[lag], acc[q]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < RG; ++q) {
+            int r = r0 + q;
+            if (r < U) p.out[r] = a.overwrite ? acc[q] : p.out[r] + acc[q];
+        }
+    }
+}
+
+// ----------------------------------------------------------------- shared-memory FFT
+// In-place Stockham autosort FFT (forward, e^{-2 pi i k m / N}) of N = 2^LOGN
+// complex values in shared memory, radix-4 passes plus one radix-2 pass when LOGN
+// is odd.  Pass with sub-transform size Ns: butterfly j reads X[j + r N/R], applies
+// twiddle W_{Ns R}^{r (j mod Ns)}, does an R-point DFT and writes output m to
+// X[(j - j mod Ns) R + j mod Ns + m Ns].  All reads of a pass complete before any
+// write (barrier), so one buffer suffices.
+template <int R>
+__device__ __forceinline__ void dft_small(float2* v) {
+    if (R == 2) {
+        float2 a = v[0], b = v[1];
+        v[0] = cadd(a, b);
+        v[1] = csub(a, b);
+    } else {  // R == 4, W_4 = -i
+        float2 s02 = cadd(v[0], v[2]), d02 = csub(v[0], v[2]);
+        float2 s13 = cadd(v[1], v[3]), d13 = csub(v[1], v[3]);
+        v[0] = cadd(s02, s13);
+        v[2] = csub(s02, s13);
+        // -i * d13 = (d13.y, -d13.x)
+        v[1] = make_float2(d02.x + d13.y, d02.y - d13.x);
+        v[3] = make_float2(d02.x - d13.y, d02.y + d13.x);
+    }
+}
+
+template <int LOGN, int NT, int R, int LOGR>
+__device__ __forceinline__ void stockham_pass(float2* X, int logNs, const float2* __restrict__ tw,
+                                              int twlog) {
+    constexpr int N = 1 << LOGN;
+    constexpr int NB = N / R;
+    constexpr int J = (NB + NT - 1) / NT;
+    const int Ns = 1 << logNs;
+    float2 v[J][R];
+#pragma unroll
+    for (int jj = 0; jj < J; ++jj) {
+        const int j = threadIdx.x + jj * NT;
+        if (j < NB) {
+            const int k = j & (Ns - 1);
+#pragma unroll
+            for (int r = 0; r < R; ++r) v[jj][r] = X[j + r * NB];
+            if (Ns > 1) {
+                const int sh = twlog - logNs - LOGR;
+#pragma unroll
+                for (int r = 1; r < R; ++r) v[jj][r] = cmul(v[jj][r], __ldg(&tw[(r * k) << sh]));
+            }
+            dft_small<R>(v[jj]);
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int jj = 0; jj < J; ++jj) {
+        const int j = threadIdx.x + jj * NT;
+        if (j < NB) {
+            const int k = j & (Ns - 1);
+            const int base = (j - k) * R + k;
+#pragma unroll
+            for (int m = 0; m < R; ++m) X[base + m * Ns] = v[jj][m];
+        }
+    }
+    __syncthreads();
+}
+
+template <int LOGN, int NT>
+__device__ __forceinline__ void fft_smem(float2* X, const float2* __restrict__ tw, int twlog) {
+    int logNs = 0;
+#pragma unroll
+    for (int p = 0; p < LOGN / 2; ++p) {
+        stockham_pass<LOGN, NT, 4, 2>(X, logNs, tw, twlog);
+        logNs += 2;
+    }
+    if (LOGN & 1) stockham_pass<LOGN, NT, 2, 1>(X, logNs, tw, twlog);
+}
+
+// Real-signal helpers.  A real sequence x of length 2N is packed as z[m] = x[2m] +
+// i x[2m+1] (m < N).  With Z = DFT_N(z), E[k] = (Z[k] + conj Z[N-k]) / 2 and
+// O[k] = (Z[k] - conj Z[N-k]) / (2i) are the DFTs of the even and odd samples, and
+// X[k] = E[k] + W^k O[k], X[k+N] = E[k] - W^k O[k] with W = e^{-2 pi i / 2N}.
+// unpack_pair returns X[k] and X[N-k] (X[N] when k = 0).
+__device__ __forceinline__ void unpack_pair(float2 Zk, float2 Zn, float2 Wk, float2 Wnk, bool k0,
+                                            float2& Xk, float2& Xn) {
+    float2 E = make_float2(0.5f * (Zk.x + Zn.x), 0.5f * (Zk.y - Zn.y));
+    float2 Dd = make_float2(Zk.x - Zn.x, Zk.y + Zn.y);  // Z[k] - conj Z[N-k]
+    float2 O = make_float2(0.5f * Dd.y, -0.5f * Dd.x);   // D / (2i)
+    Xk = cadd(E, cmul(Wk, O));
+    if (k0) Xn = make_float2(E.x - O.x, E.y - O.y);      // X[N] = E[0] - O[0]
+    else Xn = cadd(conjf2(E), cmul(Wnk, conjf2(O)));    // E[N-k] = conj E[k], same for O
+}
+// Inverse of the packing: from Y[k] and Y[N-k] of a real 2N-point signal y, the
+// values Z'[k] = E'[k] + i O'[k] with E'[k] = (Y[k] + conj Y[N-k]) / 2 and
+// O'[k] = (Y[k] - conj Y[N-k]) W^{-k} / 2, so that IDFT_N(Z')[m] = y[2m] + i y[2m+1].
+__device__ __forceinline__ float2 repack(float2 Yk, float2 Yn, float2 Wk) {
+    float2 E = make_float2(0.5f * (Yk.x + Yn.x), 0.5f * (Yk.y - Yn.y));
+    float2 Q = make_float2(0.5f * (Yk.x - Yn.x), 0.5f * (Yk.y + Yn.y));
+    float2 O = cmul(Q, conjf2(Wk));
+    return make_float2(E.x - O.y, E.y + O.x);  // E + i O
+}
+
+// Twiddle e^{-2 pi i k / 2N} from the table e^{-2 pi i m / 2^twlog}.
+template <int LOGN>
+__device__ __forceinline__ float2 tw2n(const float2* __restrict__ tw, int twlog, int k) {
+    return __ldg(&tw[k << (twlog - LOGN - 1)]);
+}
+
+// After the forward FFT of a packed, half-zero block (X = Z), form Y = X (.) H and
+// store conj of the repacked Z' so that a second forward FFT gives N conj(z').
+template <int LOGN, int NT>
+__device__ __forceinline__ void spectral_multiply(float2* X, const float2* __restrict__ H,
+                                                  const float2* __restrict__ tw, int twlog) {
+    constexpr int N = 1 << LOGN;
+    for (int k = threadIdx.x; k <= N / 2; k += NT) {
+        const int kn = (N - k) & (N - 1);
+        float2 Zk = X[k], Zn = X[kn];
+        float2 Wk = tw2n<LOGN>(tw, twlog, k);
+        float2 Wnk = tw2n<LOGN>(tw, twlog, N - k);
+        float2 Xk, Xn;
+        unpack_pair(Zk, Zn, Wk, Wnk, k == 0, Xk, Xn);
+        float2 Yk = cmul(Xk, __ldg(&H[k]));
+        float2 Yn = cmul(Xn, __ldg(&H[N - k]));
+        float2 Zpk = repack(Yk, Yn, Wk);
+        X[k] = conjf2(Zpk);
+        if (k != 0 && kn != k) {
+            float2 Zpn = repack(Yn, Yk, Wnk);
+            X[kn] = conjf2(Zpn);
+        }
+    }
+    __syncthreads();
+}
+
+// Write outputs [U, 2U-1] of the circular convolution (U = N): after the second
+// forward FFT, F = N conj(z'), so y[2m] = Re F[m] / N and y[2m+1] = -Im F[m] / N.
+template <int LOGN, int NT>
+__device__ __forceinline__ void store_upper_half(const float2* X, float* out, int overwrite) {
+    constexpr int N = 1 << LOGN;
+    const float inv = 1.0f / (float)N;
+    float2* o2 = reinterpret_cast<float2*>(out);
+    for (int m = N / 2 + threadIdx.x; m < N; m += NT) {
+        float2 F = X[m];
+        float2 v = make_float2(F.x * inv, -F.y * inv);
+        const int q = m - N / 2;
+        if (overwrite) o2[q] = v;
+        else {
+            float2 old = o2[q];
+            o2[q] = make_float2(old.x + v.x, old.y + v.y);
+        }
+    }
+}
+
+// Load a block of U = N floats as N/2 packed complex values followed by N/2 zeros.
+template <int LOGN, int NT>
+__device__ __forceinline__ void load_half_zero(float2* X, const float* in) {
+    constexpr int N = 1 << LOGN;
+    const float2* i2 = reinterpret_cast<const float2*>(in);
+    for (int m = threadIdx.x; m < N / 2; m += NT) X[m] = i2[m];
+    for (int m = N / 2 + threadIdx.x; m < N; m += NT) X[m] = make_float2(0.f, 0.f);
+    __syncthreads();
+}
+
+// ----------------------------------------------------------------- fused FFT tau
+// One gray block per CTA: rFFT_{2U}([block, 0^U]) (.) H_U -> irFFT -> outputs [U, 2U-1]
+// added onto the next U positions.  N = U complex points in shared memory.
+template <int LOGN, int NT>
+__global__ void __launch_bounds__(NT) k_tile_fft(TileArgs a) {
+    extern __shared__ float2 X[];
+    TilePtrs p = tile_ptrs(a, blockIdx.x);
+    load_half_zero<LOGN, NT>(X, p.in);
+    fft_smem<LOGN, NT>(X, a.tw, a.twlog);
+    spectral_multiply<LOGN, NT>(X, p.spec, a.tw, a.twlog);
+    fft_smem<LOGN, NT>(X, a.tw, a.twlog);
+    store_upper_half<LOGN, NT>(X, p.out, a.overwrite);
+}
+
+// ----------------------------------------------------------------- split FFT tau
+// Blocks too large for one CTA's shared memory (U = nsub * S, S = 2^LOGS): the U x U
+// block is cut into nsub x nsub sub-blocks of edge S.  Sub-block (i -> o) is the
+// same tau with its lags shifted by (o - i) S, i.e. a 2S circular convolution
+// against the spectrum of taps [e S, e S + 2S) with e = o - i + nsub - 1.  The
+// spectra of the nsub input sub-blocks are kept in a per-CTA scratch area (global
+// memory, read back by the same CTA), the products are summed in the frequency
+// domain, and one inverse FFT per output sub-block finishes it.
+template <int LOGS, int NT>
+__global__ void __launch_bounds__(NT) k_tile_fft_split(TileArgs a) {
+    extern __shared__ float2 X[];
+    constexpr int S = 1 << LOGS;
+    const int nsub = a.nsub;
+    float2* scr = a.scratch + (long long)blockIdx.x * nsub * (S + 1);
+    for (long long item = blockIdx.x; item < a.count; item += gridDim.x) {
+        TilePtrs p = tile_ptrs(a, item);
+        // spectra of the input sub-blocks
+        for (int i = 0; i < nsub; ++i) {
+            load_half_zero<LOGS, NT>(X, p.in + (long long)i * S);
+            fft_smem<LOGS, NT>(X, a.tw, a.twlog);
+            float2* Xi = scr + (long long)i * (S + 1);
+            for (int k = threadIdx.x; k <= S / 2; k += NT) {
+                const int kn = (S - k) & (S - 1);
+                float2 Xk, Xn;
+                unpack_pair(X[k], X[kn], tw2n<LOGS>(a.tw, a.twlog, k),
+                            tw2n<LOGS>(a.tw, a.twlog, S - k), k == 0, Xk, Xn);
+                Xi[k] = Xk;
+                Xi[S - k] = Xn;
+            }
+            __syncthreads();
+        }
+        // output sub-blocks
+        for (int o = 0; o < nsub; ++o) {
+            for (int k = threadIdx.x; k <= S / 2; k += NT) {
+                const int kn = (S - k) & (S - 1);
+                float2 Yk = make_float2(0.f, 0.f), Yn = make_float2(0.f, 0.f);
+                for (int i = 0; i < nsub; ++i) {
+                    const float2* Xi = scr + (long long)i * (S + 1);
+                    const float2* H = p.spec + (long long)(o - i + nsub - 1) * (S + 1);
+                    float2 hk = __ldg(&H[k]), hn = __ldg(&H[S - k]);
+                    float2 xk = Xi[k], xn = Xi[S - k];
+                    Yk = cadd(Yk, cmul(xk, hk));
+                    Yn = cadd(Yn, cmul(xn, hn));
+                }
+                float2 Wk = tw2n<LOGS>(a.tw, a.twlog, k);
+                float2 Wnk = tw2n<LOGS>(a.tw, a.twlog, S - k);
+                X[k] = conjf2(repack(Yk, Yn, Wk));
+                if (k != 0 && kn != k) X[kn] = conjf2(repack(Yn, Yk, Wnk));
+            }
+            __syncthreads();
+            fft_smem<LOGS, NT>(X, a.tw, a.twlog);
+            store_upper_half<LOGS, NT>(X, p.out + (long long)o * S, a.overwrite);
+            __syncthreads();
+        }
+    }
+}
+
+// ----------------------------------------------------------------- filter spectra
+// H[k] = sum_{m<2N} taps[off + m] e^{-2 pi i k m / 2N}, k = 0..N, for every
+// (layer, channel) item and every offset e (off = e * offstep).  Run once when a
+// context is created (section "Speicheroptimierung": DFT of the filters per block size).
+template <int LOGN, int NT>
+__global__ void __launch_bounds__(NT) k_spectra(const float* __restrict__ taps, long long ld,
+                                                int nspec, long long offstep, float2* spec,
+                                                const float2* __restrict__ tw, int twlog) {
+    extern __shared__ float2 X[];
+    constexpr int N = 1 << LOGN;
+    const long long item = blockIdx.x / nspec;
+    const int e = blockIdx.x % nspec;
+    const float2* t2 = reinterpret_cast<const float2*>(taps + item * ld + e * offstep);
+    for (int m = threadIdx.x; m < N; m += NT) X[m] = t2[m];
+    __syncthreads();
+    fft_smem<LOGN, NT>(X, tw, twlog);
+    float2* H = spec + ((long long)blockIdx.x) * (N + 1);
+    for (int k = threadIdx.x; k <= N / 2; k += NT) {
+        const int kn = (N - k) & (N - 1);
+        float2 Xk, Xn;
+        unpack_pair(X[k], X[kn], tw2n<LOGN>(tw, twlog, k), tw2n<LOGN>(tw, twlog, N - k), k == 0,
+                    Xk, Xn);
+        H[k] = Xk;
+        H[N - k] = Xn;
+    }
+}
+
+// ----------------------------------------------------------------- per-token step
+// The pages' per-token order (Algorithm 2 with Algorithm 3's layer parallelism):
+// red cells of token t for every layer in order (block and sampler = tanh), then,
+// when the released block is small, the gray block of every layer in the same
+// launch.  One lane per chain; 32 chains per CTA.
+struct StepArgs {
+    float* act;
+    const float* h;
+    int M, D;
+    long long L, G;
+    long long t;
+    const float* x;  // [G] token t, or null: take act[0][g][t]
+    float* y;        // [G] y^M_t
+    int closed;      // write a^M_t as token t+1
+    int fuseU;       // edge of the block n = t+1 done here (0: none)
+};
+
+template <int NT>
+__global__ void __launch_bounds__(NT) k_token_step(StepArgs a) {
+    const long long g0 = (long long)blockIdx.x * 32;
+    const int lane = threadIdx.x;
+    const long long t = a.t;
+    if (lane < 32) {
+        const long long g = g0 + lane;
+        if (g < a.G) {
+            const long long c = g % a.D;
+            float av = a.x ? a.x[g] : a.act[g * a.L + t];
+            a.act[g * a.L + t] = av;
+            float y = 0.f;
+            for (int l = 1; l <= a.M; ++l) {
+                float* slot = a.act + ((long long)l * a.G + g) * a.L + t;
+                const float h0 = a.h[((long long)(l - 1) * a.D + c) * a.L];
+                const float p = (t == 0) ? 0.f : *slot;
+                y = fmaf(h0, av, p);
+                av = act_tanh(y);
+                *slot = av;
+            }
+            a.y[g] = y;
+            if (a.closed && t + 1 < a.L) a.act[g * a.L + t + 1] = av;
+        }
+    }
+    const int U = a.fuseU;
+    if (U == 0) return;
+    __syncthreads();
+    const long long n = t + 1;
+    const bool ow = is_pow2(n);
+    const int nch = (int)min(32LL, a.G - g0);
+    const int items = nch * a.M * U;
+    for (int it = threadIdx.x; it < items; it += NT) {
+        const int r = it % U;
+        const int rest = it / U;
+        const int i = rest % nch;
+        const int l = rest / nch + 1;
+        const long long g = g0 + i;
+        const long long c = g % a.D;
+        const float* in = a.act + ((long long)(l - 1) * a.G + g) * a.L + (n - U);
+        const float* hp = a.h + ((long long)(l - 1) * a.D + c) * a.L + U + r;
+        float acc = 0.f;
+        for (int j = 0; j < U; ++j) acc = fmaf(in[j], hp[-j], acc);
+        float* o = a.act + ((long long)l * a.G + g) * a.L + n + r;
+        *o = ow ? acc : *o + acc;
+    }
+}
+
+// ----------------------------------------------------------------- window kernel
+// Persistent per-window kernel (the B200 form of the per-token CUDA graph): one
+// CTA holds `kch` channels x B batch rows ("chains") and runs tokens [t0, t1) of one
+// aligned window [kW, kW+W) entirely in shared memory.  Every block of edge U < W
+// released inside the window reads and writes only positions of that window (n =
+// kW + m with 0 < m < W, U = lowbit(m): [n-U, n+U-1] lies in the window), so the
+// window is self-contained; blocks of edge >= W are released only at window ends
+// and run as separate launches over all chains.
+//
+// Work split inside a step (token t, window offset s):
+//  * chain lanes (warp 0, one lane per chain): the red cells of all layers, in
+//    order, plus the one term of row 0 of block n = t that needs a^{l-1}_{t-1}.
+//  * helper warps, concurrently: rows 1..U-1 of block n = t, and row 0 of block
+//    n = t+1 without its newest input (all its inputs are older than t).
+// Rows of a block are needed one token after the other, so this keeps every
+// block off the chain lanes' critical path except one multiply-add per layer.
+// The launch's first token skips the work of block n = t0 (it is complete: the
+// previous launch or the large-block launch finished it), and a launch that ends
+// inside a window completes block n = t1 before storing, so the buffers in global
+// memory always hold the state the per-token path expects.
+struct WinArgs {
+    float* act;
+    const float* h;
+    int M, B, D;
+    long long L, G;
+    long long t0, t1;   // tokens of this launch (one window)
+    long long tx;       // token of x[0] / out[0]
+    const float* x;     // teacher: [.][G] tokens; closed loop: [G] token t0 or null
+    float* out;         // [.][G] y^M
+    int closed;
+    int kch;            // channels per CTA
+};
+
+template <int W>
+struct WinSmem {
+    static constexpr int P = W + 1;  // padded row pitch: lanes of different chains hit different banks
+};
+
+// rows 1..U-1 of the block released after token t (window offset s, U = lowbit(s))
+template <int W>
+__device__ __forceinline__ void win_rows(float* slot, const float* tap, int M, int ncb, int nch,
+                                         int CPB, int kch, int s, bool ow, int ht, int nh) {
+    constexpr int P = WinSmem<W>::P;
+    constexpr int RG = 4;
+    const int U = s & (-s);
+    if (U < 2) return;
+    const int nrows = U - 1;
+    const int ngrp = (nrows + RG - 1) / RG;
+    const int items = M * ncb * ngrp;
+    for (int it = ht; it < items; it += nh) {
+        const int grp = it % ngrp;
+        const int rest = it / ngrp;
+        const int i = rest % ncb;
+        const int l = rest / ncb + 1;
+        const int ci = i % nch;
+        const float* in = slot + ((l - 1) * CPB + i) * P + (s - U);
+        const float* tp = tap + ((l - 1) * kch + ci) * P;
+        const int r0 = 1 + grp * RG;
+        float acc[RG];
+#pragma unroll
+        for (int q = 0; q < RG; ++q) acc[q] = 0.f;
+        for (int j = 0; j < U; ++j) {
+            const float xv = in[j];
+#pragma unroll
+            for (int q = 0; q < RG; ++q)
+                if (r0 + q < U) acc[q] = fmaf(xv, tp[U + r0 + q - j], acc[q]);
+        }
+        float* o = slot + (l * CPB + i) * P + s;
+#pragma unroll
+        for (int q = 0; q < RG; ++q) {
+            const int r = r0 + q;
+            if (r < U) o[r] = ow ? acc[q] : o[r] + acc[q];
+        }
+    }
+}
+
+template <int W, int NT>
+__global__ void __launch_bounds__(NT) k_window(WinArgs a) {
+    extern __shared__ float sm[];
+    constexpr int P = WinSmem<W>::P;
+    const int M = a.M, B = a.B, D = a.D, kch = a.kch;
+    const long long L = a.L, G = a.G;
+    const int c0 = blockIdx.x * kch;
+    const int nch = min(kch, D - c0);
+    const int ncb = nch * B;
+    const int CPB = kch * B;
+    float* slot = sm;                                   // [(M+1) * CPB][P]
+    float* tap = sm + (size_t)(M + 1) * CPB * P;         // [M * kch][P]
+    const long long kW = (a.t0 / W) * (long long)W;
+    const int wlen = (int)min((long long)W, L - kW);
+    const int s0 = (int)(a.t0 - kW), s1 = (int)(a.t1 - kW);
+    const int tid = threadIdx.x;
+
+    // ---- stage the window of every layer, and taps 0..W-1
+    {
+        const int per = (M + 1) * ncb;
+        for (int e = tid; e < per * wlen; e += NT) {
+            const int s = e % wlen;
+            const int rest = e / wlen;
+            const int i = rest % ncb;
+            const int l = rest / ncb;
+            const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+            slot[(l * CPB + i) * P + s] = a.act[((long long)l * G + g) * L + kW + s];
+        }
+        for (int e = tid; e < M * nch * wlen; e += NT) {
+            const int s = e % wlen;
+            const int rest = e / wlen;
+            const int ci = rest % nch;
+            const int l = rest / nch;
+            tap[(l * kch + ci) * P + s] = a.h[((long long)l * D + c0 + ci) * L + s];
+        }
+        __syncthreads();
+        if (!a.closed) {
+            const int steps = s1 - s0;
+            for (int e = tid; e < steps * ncb; e += NT) {
+                const int i = e % ncb;
+                const int s = s0 + e / ncb;
+                const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+                slot[i * P + s] = a.x[(kW + s - a.tx) * G + g];
+            }
+        } else if (a.x) {
+            for (int i = tid; i < ncb; i += NT) {
+                const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+                slot[i * P + s0] = a.x[g];
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- tokens
+    const int lane = tid;  // chain lanes: warp 0
+    const bool chain = tid < 32 && lane < ncb;
+    long long gch = 0;
+    int cich = 0;
+    if (chain) {
+        cich = lane % nch;
+        gch = (long long)(lane / nch) * D + c0 + cich;
+    }
+    const int ht = tid - 32, nh = NT - 32;
+    for (int s = s0; s < s1; ++s) {
+        const long long t = kW + s;
+        if (tid < 32) {
+            if (chain) {
+                const bool newest = s > s0;  // row 0 of block n = t still lacks a^{l-1}_{t-1}
+                const float* tp = tap + cich * P;
+                float av = slot[lane * P + s];
+                float y = 0.f;
+                // software-pipelined: fetch layer l+1's running sum before layer l's tanh
+                float pn = (t == 0) ? 0.f : slot[(1 * CPB + lane) * P + s];
+                if (newest) pn = fmaf(tp[1], slot[lane * P + s - 1], pn);
+                float h0n = tp[0];
+                for (int l = 1; l <= M; ++l) {
+                    const float p = pn, h0 = h0n;
+                    if (l < M) {
+                        const float* tq = tap + (l * kch + cich) * P;
+                        pn = (t == 0) ? 0.f : slot[((l + 1) * CPB + lane) * P + s];
+                        if (newest) pn = fmaf(tq[1], slot[(l * CPB + lane) * P + s - 1], pn);
+                        h0n = tq[0];
+                    }
+                    y = fmaf(h0, av, p);
+                    av = act_tanh(y);
+                    slot[(l * CPB + lane) * P + s] = av;
+                }
+                a.out[(t - a.tx) * G + gch] = y;
+                if (a.closed) {
+                    if (s + 1 < wlen) slot[lane * P + s + 1] = av;
+                    else if (t + 1 < L) a.act[gch * L + t + 1] = av;
+                }
+            }
+        } else {
+            // rows 1..U-1 of block n = t (its first token in this launch is complete already)
+            if (s > s0) win_rows<W>(slot, tap, M, ncb, nch, CPB, kch, s, is_pow2(t), ht, nh);
+            // row 0 of block n = t+1, all inputs except a^{l-1}_t
+            if (s + 1 < wlen) {
+                const int s1p = s + 1;
+                const int U1 = s1p & (-s1p);
+                const bool ow1 = is_pow2(t + 1);
+                if (U1 >= 2 || ow1) {
+                    for (int it = ht; it < M * ncb; it += nh) {
+                        const int i = it % ncb;
+                        const int l = it / ncb + 1;
+                        const float* in = slot + ((l - 1) * CPB + i) * P + (s1p - U1);
+                        const float* tp = tap + ((l - 1) * kch + (i % nch)) * P;
+                        float acc = 0.f;
+                        for (int j = 0; j < U1 - 1; ++j) acc = fmaf(in[j], tp[U1 - j], acc);
+                        float* o = slot + (l * CPB + i) * P + s1p;
+                        *o = ow1 ? acc : *o + acc;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---- a launch that stops inside the window completes block n = t1
+    if (s1 < wlen && s1 > s0) {
+        const long long n = kW + s1;
+        if (chain) {
+            for (int l = 1; l <= M; ++l) {
+                const float* tp = tap + ((l - 1) * kch + cich) * P;
+                float* o = slot + (l * CPB + lane) * P + s1;
+                *o = fmaf(tp[1], slot[((l - 1) * CPB + lane) * P + s1 - 1], *o);
+            }
+        }
+        if (tid >= 32) win_rows<W>(slot, tap, M, ncb, nch, CPB, kch, s1, is_pow2(n), ht, nh);
+        __syncthreads();
+    }
+
+    // ---- write the window back (positions >= t0 of every layer)
+    {
+        const int span = wlen - s0;
+        const int per = (M + 1) * ncb;
+        for (int e = tid; e < per * span; e += NT) {
+            const int s = s0 + e % span;
+            const int rest = e / span;
+            const int i = rest % ncb;
+            const int l = rest / ncb;
+            const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+            a.act[((long long)l * G + g) * L + kW + s] = slot[(l * CPB + i) * P + s];
+        }
+    }
+}
+
+// ----------------------------------------------------------------- read-out
+// dst[(t - t0) * G + g] = act[layer][g][t] for t in [t0, t1)
+__global__ void k_read_layer(const float* __restrict__ act, long long L, long long G, int layer,
+                             long long t0, long long t1, float* dst) {
+    const long long total = (t1 - t0) * G;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const long long g = e % G;
+        const long long t = t0 + e / G;
+        dst[e] = act[((long long)layer * G + g) * L + t];
+    }
+}
+
+}  // namespace fi
