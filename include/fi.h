@@ -98,6 +98,8 @@ typedef struct fi_trace {
     int launches[FI_K_CLASSES];     /* launches of each class in the last run */
     double total_us[FI_K_CLASSES];  /* summed device time of those launches */
     double max_us[FI_K_CLASSES];    /* longest single launch */
+    int block_launches[32];         /* block launches of edge 2^q */
+    double block_us[32];            /* their summed device time */
 } fi_trace;
 
 /* Create a context for `layers` stacked mixers over B sequences of D channels,

@@ -38,7 +38,8 @@ KERNEL_CLASS_NAMES = ("window", "token_step", "block_direct", "block_fft", "bloc
 
 class fi_trace(ctypes.Structure):
     _fields_ = [("launches", ctypes.c_int * FI_K_CLASSES), ("total_us", ctypes.c_double * FI_K_CLASSES),
-                ("max_us", ctypes.c_double * FI_K_CLASSES)]
+                ("max_us", ctypes.c_double * FI_K_CLASSES),
+                ("block_launches", ctypes.c_int * 32), ("block_us", ctypes.c_double * 32)]
 
 
 # Every entry point declared in include/fi.h, with its C signature.
@@ -171,12 +172,16 @@ class FlashInference:
     def set_trace(self, on: bool):
         _check(get_lib().fi_set_trace(self._h, int(bool(on))))
 
-    def trace(self) -> dict:
-        """{class name: (launches, total_us, max_us)} of the last traced run."""
+    def trace(self, per_block_size: bool = False):
+        """{class name: (launches, total_us, max_us)} of the last traced run; with
+        per_block_size also {q: (launches, total_us)} of the block launches."""
         tr = fi_trace()
         _check(get_lib().fi_trace_read(self._h, ctypes.byref(tr)))
-        return {KERNEL_CLASS_NAMES[k]: (tr.launches[k], tr.total_us[k], tr.max_us[k])
-                for k in range(FI_K_CLASSES) if tr.launches[k]}
+        cls = {KERNEL_CLASS_NAMES[k]: (tr.launches[k], tr.total_us[k], tr.max_us[k])
+               for k in range(FI_K_CLASSES) if tr.launches[k]}
+        if not per_block_size:
+            return cls
+        return cls, {q: (tr.block_launches[q], tr.block_us[q]) for q in range(32) if tr.block_launches[q]}
 
     def info(self) -> fi_info:
         inf = fi_info()

@@ -56,7 +56,6 @@ constexpr int kLogSMax = 14;        // largest FFT held by one CTA: 2^14 complex
 constexpr int kFftQMin = 3;         // smallest block size served by FFT (U = 8)
 constexpr int kDirectQMax = 12;     // largest block size served by the direct kernel
 constexpr int kFuseQMax = 4;        // per-token path: blocks up to U = 16 run inside the step kernel
-constexpr int kWinNT = 256;         // threads of the window kernel (1 chain warp + 7 helper warps)
 constexpr int kStepNT = 128;
 constexpr int kDirectNT = 128;
 constexpr size_t kSmemMax = 227 * 1024;
@@ -74,6 +73,7 @@ struct GraphKey {
 
 struct TraceRec {
     int cls;
+    int q;  // block size 2^q of block launches, -1 otherwise
     cudaEvent_t a, b;
 };
 
@@ -170,10 +170,12 @@ struct LaunchScope {
     cudaStream_t st;
     TraceRec r;
     bool on;
-    LaunchScope(fi_ctx* c_, int cls, cudaStream_t st_) : c(c_), st(st_), on(c_->trace_on && c_->rec) {
+    LaunchScope(fi_ctx* c_, int cls, cudaStream_t st_, int q = -1)
+        : c(c_), st(st_), on(c_->trace_on && c_->rec) {
         c->enq_launches++;
         if (on) {
             r.cls = cls;
+            r.q = q;
             r.a = pool_event(c);
             r.b = pool_event(c);
             on = r.a && r.b;
@@ -205,8 +207,11 @@ int dev_alloc(fi_ctx* c, T** p, size_t count) {
 }
 
 size_t win_smem_bytes(int W, int M, int B, int kch) {
-    return (size_t)((M + 1) * kch * B + M * kch) * (W + 1) * sizeof(float);
+    return (size_t)((M + 1) * kch * B + M * kch) * (W + 2) * sizeof(float);
 }
+
+// chain registers of the window kernel are unrolled up to MAXM layers
+int win_maxm(int M) { return M <= 8 ? 8 : (M <= 20 ? 20 : (M <= 40 ? 40 : 0)); }
 
 // ---------------------------------------------------------------- kernel launchers
 template <int LOGN>
@@ -281,20 +286,29 @@ int launch_spectra(int logn, const float* taps, long long ld, int count, int nsp
     }
 }
 
-template <int W>
+template <int W, int MAXM>
 int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
-    k_window<W, kWinNT><<<c->win_ncta, kWinNT, c->win_smem, st>>>(a);
+    k_window<W, MAXM><<<c->win_ncta, kWinThreads, c->win_smem, st>>>(a);
     CK(cudaGetLastError());
     return FI_OK;
 }
 
+template <int W>
+int launch_window_w(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
+    switch (win_maxm(c->M)) {
+        case 8: return launch_window_t<W, 8>(c, a, st);
+        case 20: return launch_window_t<W, 20>(c, a, st);
+        case 40: return launch_window_t<W, 40>(c, a, st);
+        default: return set_err(FI_EINVAL, "window kernel supports at most 40 layers");
+    }
+}
+
 int launch_window(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
     switch (c->W) {
-        case 16: return launch_window_t<16>(c, a, st);
-        case 32: return launch_window_t<32>(c, a, st);
-        case 64: return launch_window_t<64>(c, a, st);
-        case 128: return launch_window_t<128>(c, a, st);
-        case 256: return launch_window_t<256>(c, a, st);
+        case 32: return launch_window_w<32>(c, a, st);
+        case 64: return launch_window_w<64>(c, a, st);
+        case 128: return launch_window_w<128>(c, a, st);
+        case 256: return launch_window_w<256>(c, a, st);
         default: return set_err(FI_EINVAL, "unsupported window %d", c->W);
     }
 }
@@ -310,22 +324,26 @@ int attr_fft() {
     return FI_OK;
 }
 
+template <int W>
+int attr_window() {
+    CK(cudaFuncSetAttribute(k_window<W, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 20>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 40>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    return FI_OK;
+}
+
 int set_all_attrs() {
     static int done = 0;
     if (done) return FI_OK;
     int rc = 0;
     rc |= attr_fft<3>() | attr_fft<4>() | attr_fft<5>() | attr_fft<6>() | attr_fft<7>() | attr_fft<8>();
     rc |= attr_fft<9>() | attr_fft<10>() | attr_fft<11>() | attr_fft<12>() | attr_fft<13>() | attr_fft<14>();
+    rc |= attr_window<32>() | attr_window<64>() | attr_window<128>() | attr_window<256>();
     if (rc) return FI_ECUDA;
     CK(cudaFuncSetAttribute(k_tile_fft_split<kLogSMax, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                             (int)(sizeof(float2) << kLogSMax)));
     CK(cudaFuncSetAttribute(k_tile_direct<kDirectNT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                             (int)(3 * (1 << kDirectQMax) * sizeof(float))));
-    CK(cudaFuncSetAttribute(k_window<16, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<32, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<64, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<128, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<256, kWinNT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
     done = 1;
     return FI_OK;
 }
@@ -354,7 +372,7 @@ int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st) {
     const int q = ctz64(n);
     const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
                     : (c->spec_split[q] > 1 ? FI_K_BLOCK_SPLIT : FI_K_BLOCK_FFT);
-    LaunchScope scope(c, cls, st);
+    LaunchScope scope(c, cls, st, q);
     if (impl == FI_TAU_DIRECT) return launch_direct_tile(a, st);
     a.spec = c->spec[q];
     a.spec_stride = c->spec_stride[q];
@@ -594,7 +612,8 @@ int choose_window(fi_ctx* c) {
     if (kch * c->B > 32) kch = std::max(1, 32 / c->B);
     const int ncta = (c->D + kch - 1) / kch;
     const int per_sm = (ncta + c->nsm - 1) / c->nsm;
-    const int cand[] = {256, 128, 64, 32, 16};
+    if (!win_maxm(c->M)) return FI_OK;
+    const int cand[] = {256, 128, 64, 32};
     for (int W : cand) {
         if (forced && W != forced) continue;
         if (W > c->L) continue;
@@ -946,6 +965,10 @@ int fi_trace_read(fi_ctx* ctx, fi_trace* out) {
         out->launches[r.cls] += 1;
         out->total_us[r.cls] += 1000.0 * ms;
         if (1000.0 * ms > out->max_us[r.cls]) out->max_us[r.cls] = 1000.0 * ms;
+        if (r.q >= 0 && r.q < 32) {
+            out->block_launches[r.q] += 1;
+            out->block_us[r.q] += 1000.0 * ms;
+        }
     }
     return FI_OK;
 }

@@ -480,17 +480,20 @@ __global__ void __launch_bounds__(NT) k_token_step(StepArgs a) {
 // window is self-contained; blocks of edge >= W are released only at window ends
 // and run as separate launches over all chains.
 //
-// Work split inside a step (token t, window offset s):
-//  * chain lanes (warp 0, one lane per chain): the red cells of all layers, in
-//    order, plus the one term of row 0 of block n = t that needs a^{l-1}_{t-1}.
-//  * helper warps, concurrently: rows 1..U-1 of block n = t, and row 0 of block
-//    n = t+1 without its newest input (all its inputs are older than t).
-// Rows of a block are needed one token after the other, so this keeps every
-// block off the chain lanes' critical path except one multiply-add per layer.
-// The launch's first token skips the work of block n = t0 (it is complete: the
-// previous launch or the large-block launch finished it), and a launch that ends
-// inside a window completes block n = t1 before storing, so the buffers in global
-// memory always hold the state the per-token path expects.
+// Inside the window every block row is evaluated one token before it is needed:
+//  * chain lanes (warp 0, one lane per chain) run the red cells of all layers in
+//    order, plus the single term of row 0 of block n = t that needs a^{l-1}_{t-1};
+//  * helper warps, concurrently, finish position T = t+1: they add the rows of the
+//    blocks n in (t0, T] that cover T, except that newest term.  Walking n = T,
+//    T - lowbit(T), ... (each step clears the lowest set bit) lists exactly those
+//    blocks; their input ranges are adjacent, so the rows form one dot product over
+//    inputs [lo, t-1] per (layer, chain).
+// A block is therefore never computed as a burst on the chain's critical path, and
+// each step costs one barrier.  Blocks released at or before t0 were completed by
+// the previous launch (or by the large-block launch at a window start); a launch
+// that stops inside the window completes the blocks it released before storing, so
+// the buffers always hold the state the per-token path expects: every block
+// n <= t applied.
 struct WinArgs {
     float* act;
     const float* h;
@@ -504,53 +507,72 @@ struct WinArgs {
     int kch;            // channels per CTA
 };
 
-template <int W>
-struct WinSmem {
-    static constexpr int P = W + 1;  // padded row pitch: lanes of different chains hit different banks
-};
+constexpr int kWinThreads = 256;          // warp 0: chain lanes; warps 1..7: helpers
+constexpr int kWinPairs = (kWinThreads - 32) / 2;
 
-// rows 1..U-1 of the block released after token t (window offset s, U = lowbit(s))
-template <int W>
-__device__ __forceinline__ void win_rows(float* slot, const float* tap, int M, int ncb, int nch,
-                                         int CPB, int kch, int s, bool ow, int ht, int nh) {
-    constexpr int P = WinSmem<W>::P;
-    constexpr int RG = 4;
-    const int U = s & (-s);
-    if (U < 2) return;
-    const int nrows = U - 1;
-    const int ngrp = (nrows + RG - 1) / RG;
-    const int items = M * ncb * ngrp;
-    for (int it = ht; it < items; it += nh) {
-        const int grp = it % ngrp;
-        const int rest = it / ngrp;
-        const int i = rest % ncb;
-        const int l = rest / ncb + 1;
-        const int ci = i % nch;
-        const float* in = slot + ((l - 1) * CPB + i) * P + (s - U);
-        const float* tp = tap + ((l - 1) * kch + ci) * P;
-        const int r0 = 1 + grp * RG;
-        float acc[RG];
-#pragma unroll
-        for (int q = 0; q < RG; ++q) acc[q] = 0.f;
-        for (int j = 0; j < U; ++j) {
-            const float xv = in[j];
-#pragma unroll
-            for (int q = 0; q < RG; ++q)
-                if (r0 + q < U) acc[q] = fmaf(xv, tp[U + r0 + q - j], acc[q]);
+// Lowest input of the blocks released at n in (s0, hi] that cover window position T
+// (window-local), walking n = T, T - lowbit(T), ...; returns -1 if none.  *top gets
+// the highest such input (the first covering block released at or before hi).
+__device__ __forceinline__ int cover_range(int T, int s0, int hi, int* top) {
+    int lo = -1, n = T;
+    *top = -1;
+    while (n > s0 && n > 0) {
+        const int lon = n - (n & (-n));
+        if (n <= hi) {
+            if (*top < 0) *top = n - 1;
+            lo = lon;
         }
-        float* o = slot + (l * CPB + i) * P + s;
-#pragma unroll
-        for (int q = 0; q < RG; ++q) {
-            const int r = r0 + q;
-            if (r < U) o[r] = ow ? acc[q] : o[r] + acc[q];
+        n = lon;
+    }
+    return lo;
+}
+
+// sum over j = jb, jb+2, ... < je of in[j] * tp[T - j]
+__device__ __forceinline__ float dot_stride2(const float* in, const float* tp, int T, int jb, int je) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int j = jb;
+    for (; j + 6 < je; j += 8) {
+        a0 = fmaf(in[j], tp[T - j], a0);
+        a1 = fmaf(in[j + 2], tp[T - j - 2], a1);
+        a2 = fmaf(in[j + 4], tp[T - j - 4], a2);
+        a3 = fmaf(in[j + 6], tp[T - j - 6], a3);
+    }
+    for (; j < je; j += 2) a0 = fmaf(in[j], tp[T - j], a0);
+    return (a0 + a1) + (a2 + a3);
+}
+
+// Helper pairs add the rows over inputs [lo, hi] onto position T of every
+// (layer, chain); overwrite when these rows include the position's first writer.
+template <int P>
+__device__ __forceinline__ void helper_rows(float* slot, const float* tap, int M, int ncb, int nch, int CPB,
+                                            int kch, int T, int lo, int hi, bool ow, int pair, int part) {
+    const int items = M * ncb;
+    for (int base = 0; base < items; base += kWinPairs) {
+        const int it = base + pair;
+        float acc = 0.f;
+        int l = 0, i = 0;
+        if (it < items) {
+            l = it / ncb + 1;
+            i = it - (l - 1) * ncb;
+            const float* in = slot + ((l - 1) * CPB + i) * P;
+            const float* tp = tap + ((l - 1) * kch + (i % nch)) * P;
+            acc = dot_stride2(in, tp, T, lo + part, hi + 1);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (it < items && part == 0) {
+            float* o = slot + (l * CPB + i) * P + T;
+            *o = ow ? acc : *o + acc;
         }
     }
 }
 
-template <int W, int NT>
-__global__ void __launch_bounds__(NT) k_window(WinArgs a) {
-    extern __shared__ float sm[];
-    constexpr int P = WinSmem<W>::P;
+template <int W, int MAXM>
+__global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
+    extern __shared__ float4 sm4[];
+    float* sm = reinterpret_cast<float*>(sm4);
+    constexpr int NT = kWinThreads;
+    constexpr int P = W + 2;  // row pitch: the two lanes of a helper pair and consecutive rows hit distinct banks
+    constexpr float K = 2.8853900817779268f;  // 2 / ln 2: tanh(y) = 1 - 2 / (1 + 2^(K y))
     const int M = a.M, B = a.B, D = a.D, kch = a.kch;
     const long long L = a.L, G = a.G;
     const int c0 = blockIdx.x * kch;
@@ -559,28 +581,49 @@ __global__ void __launch_bounds__(NT) k_window(WinArgs a) {
     const int CPB = kch * B;
     float* slot = sm;                                   // [(M+1) * CPB][P]
     float* tap = sm + (size_t)(M + 1) * CPB * P;         // [M * kch][P]
-    const long long kW = (a.t0 / W) * (long long)W;
-    const int wlen = (int)min((long long)W, L - kW);
+    const long long kW = (a.t0 / W) * (long long)W;      // windows never cross L (W divides L)
     const int s0 = (int)(a.t0 - kW), s1 = (int)(a.t1 - kW);
     const int tid = threadIdx.x;
 
-    // ---- stage the window of every layer, and taps 0..W-1
+    // ---- stage the window of every layer and taps 0..W-1 (batched 16-byte loads)
     {
-        const int per = (M + 1) * ncb;
-        for (int e = tid; e < per * wlen; e += NT) {
-            const int s = e % wlen;
-            const int rest = e / wlen;
-            const int i = rest % ncb;
-            const int l = rest / ncb;
-            const long long g = (long long)(i / nch) * D + c0 + (i % nch);
-            slot[(l * CPB + i) * P + s] = a.act[((long long)l * G + g) * L + kW + s];
-        }
-        for (int e = tid; e < M * nch * wlen; e += NT) {
-            const int s = e % wlen;
-            const int rest = e / wlen;
-            const int ci = rest % nch;
-            const int l = rest / nch;
-            tap[(l * kch + ci) * P + s] = a.h[((long long)l * D + c0 + ci) * L + s];
+        constexpr int PER = W / 4;
+        const int rows_slot = (M + 1) * ncb;
+        const int total = (rows_slot + M * nch) * PER;
+        for (int e0 = tid; e0 < total; e0 += NT * 8) {
+            float4 v[8];
+            int dst[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * NT;
+                dst[u] = -1;
+                if (e < total) {
+                    const int row = e / PER, c4 = e - row * PER;
+                    const float* src;
+                    if (row < rows_slot) {
+                        const int l = row / ncb, i = row - l * ncb;
+                        const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+                        src = a.act + ((long long)l * G + g) * L + kW + 4 * c4;
+                        dst[u] = (l * CPB + i) * P + 4 * c4;
+                    } else {
+                        const int r2 = row - rows_slot;
+                        const int l = r2 / nch, ci = r2 - l * nch;
+                        src = a.h + ((long long)l * D + c0 + ci) * L + 4 * c4;
+                        dst[u] = (M + 1) * CPB * P + (l * kch + ci) * P + 4 * c4;
+                    }
+                    v[u] = __ldg(reinterpret_cast<const float4*>(src));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (dst[u] >= 0) {
+                    float* d = sm + dst[u];
+                    d[0] = v[u].x;
+                    d[1] = v[u].y;
+                    d[2] = v[u].z;
+                    d[3] = v[u].w;
+                }
+            }
         }
         __syncthreads();
         if (!a.closed) {
@@ -601,7 +644,7 @@ __global__ void __launch_bounds__(NT) k_window(WinArgs a) {
     }
 
     // ---- tokens
-    const int lane = tid;  // chain lanes: warp 0
+    const int lane = tid;
     const bool chain = tid < 32 && lane < ncb;
     long long gch = 0;
     int cich = 0;
@@ -609,87 +652,95 @@ __global__ void __launch_bounds__(NT) k_window(WinArgs a) {
         cich = lane % nch;
         gch = (long long)(lane / nch) * D + c0 + cich;
     }
-    const int ht = tid - 32, nh = NT - 32;
+    const int pair = (tid - 32) >> 1, part = tid & 1;
     for (int s = s0; s < s1; ++s) {
         const long long t = kW + s;
         if (tid < 32) {
             if (chain) {
-                const bool newest = s > s0;  // row 0 of block n = t still lacks a^{l-1}_{t-1}
-                const float* tp = tap + cich * P;
-                float av = slot[lane * P + s];
-                float y = 0.f;
-                // software-pipelined: fetch layer l+1's running sum before layer l's tanh
-                float pn = (t == 0) ? 0.f : slot[(1 * CPB + lane) * P + s];
-                if (newest) pn = fmaf(tp[1], slot[lane * P + s - 1], pn);
-                float h0n = tp[0];
-                for (int l = 1; l <= M; ++l) {
-                    const float p = pn, h0 = h0n;
-                    if (l < M) {
-                        const float* tq = tap + (l * kch + cich) * P;
-                        pn = (t == 0) ? 0.f : slot[((l + 1) * CPB + lane) * P + s];
-                        if (newest) pn = fmaf(tq[1], slot[(l * CPB + lane) * P + s - 1], pn);
-                        h0n = tq[0];
+                // running sums of every layer first (independent of the chain), then the
+                // link chain in registers: z_l = K y_l, r_l = 1 / (1 + 2^z_l), a_l = 1 - 2 r_l,
+                // z_{l+1} = (-2 K h0) r_l + (K h0 + K p_{l+1})
+                const bool newest = s > s0;
+                float c1[MAXM], c2[MAXM];
+#pragma unroll
+                for (int l = 1; l <= MAXM; ++l) {
+                    if (l <= M) {
+                        const float* tl = tap + ((l - 1) * kch + cich) * P;
+                        float p = (t == 0) ? 0.f : slot[(l * CPB + lane) * P + s];
+                        if (newest) p = fmaf(tl[1], slot[((l - 1) * CPB + lane) * P + s - 1], p);
+                        const float hs = K * tl[0];
+                        if (l == 1) {
+                            c1[0] = hs;
+                            c2[0] = K * p;
+                        } else {
+                            c1[l - 1] = -2.f * hs;
+                            c2[l - 1] = fmaf(K, p, hs);
+                        }
                     }
-                    y = fmaf(h0, av, p);
-                    av = act_tanh(y);
-                    slot[(l * CPB + lane) * P + s] = av;
                 }
-                a.out[(t - a.tx) * G + gch] = y;
+                const float a0 = slot[lane * P + s];
+                float z = fmaf(c1[0], a0, c2[0]);
+                float r = sfu_rcp(1.0f + sfu_ex2(z));
+                slot[(CPB + lane) * P + s] = fmaf(-2.f, r, 1.f);
+#pragma unroll
+                for (int l = 2; l <= MAXM; ++l) {
+                    if (l <= M) {
+                        z = fmaf(c1[l - 1], r, c2[l - 1]);
+                        r = sfu_rcp(1.0f + sfu_ex2(z));
+                        slot[(l * CPB + lane) * P + s] = fmaf(-2.f, r, 1.f);
+                    }
+                }
+                a.out[(t - a.tx) * G + gch] = z * (1.0f / K);
                 if (a.closed) {
-                    if (s + 1 < wlen) slot[lane * P + s + 1] = av;
-                    else if (t + 1 < L) a.act[gch * L + t + 1] = av;
+                    const float aM = fmaf(-2.f, r, 1.f);
+                    if (s + 1 < W) slot[lane * P + s + 1] = aM;
+                    else if (t + 1 < L) a.act[gch * L + t + 1] = aM;
                 }
             }
         } else {
-            // rows 1..U-1 of block n = t (its first token in this launch is complete already)
-            if (s > s0) win_rows<W>(slot, tap, M, ncb, nch, CPB, kch, s, is_pow2(t), ht, nh);
-            // row 0 of block n = t+1, all inputs except a^{l-1}_t
-            if (s + 1 < wlen) {
-                const int s1p = s + 1;
-                const int U1 = s1p & (-s1p);
-                const bool ow1 = is_pow2(t + 1);
-                if (U1 >= 2 || ow1) {
-                    for (int it = ht; it < M * ncb; it += nh) {
-                        const int i = it % ncb;
-                        const int l = it / ncb + 1;
-                        const float* in = slot + ((l - 1) * CPB + i) * P + (s1p - U1);
-                        const float* tp = tap + ((l - 1) * kch + (i % nch)) * P;
-                        float acc = 0.f;
-                        for (int j = 0; j < U1 - 1; ++j) acc = fmaf(in[j], tp[U1 - j], acc);
-                        float* o = slot + (l * CPB + i) * P + s1p;
-                        *o = ow1 ? acc : *o + acc;
-                    }
-                }
+            const int T = s + 1;
+            if (T < W) {
+                int top;
+                const int lo = cover_range(T, s0, T, &top);
+                helper_rows<P>(slot, tap, M, ncb, nch, CPB, kch, T, lo, s - 1, kW == 0 && lo == 0, pair, part);
             }
         }
         __syncthreads();
     }
 
-    // ---- a launch that stops inside the window completes block n = t1
-    if (s1 < wlen && s1 > s0) {
-        const long long n = kW + s1;
+    // ---- a launch that stops inside the window completes the blocks it released
+    if (s1 < W && s1 > s0) {
         if (chain) {
             for (int l = 1; l <= M; ++l) {
-                const float* tp = tap + ((l - 1) * kch + cich) * P;
+                const float* tl = tap + ((l - 1) * kch + cich) * P;
                 float* o = slot + (l * CPB + lane) * P + s1;
-                *o = fmaf(tp[1], slot[((l - 1) * CPB + lane) * P + s1 - 1], *o);
+                *o = fmaf(tl[1], slot[((l - 1) * CPB + lane) * P + s1 - 1], *o);
             }
         }
-        if (tid >= 32) win_rows<W>(slot, tap, M, ncb, nch, CPB, kch, s1, is_pow2(n), ht, nh);
+        if (tid >= 32) {
+            for (int T = s1 + 1; T < W; ++T) {
+                int top;
+                const int lo = cover_range(T, s0, s1, &top);
+                if (lo >= 0)
+                    helper_rows<P>(slot, tap, M, ncb, nch, CPB, kch, T, lo, top, kW == 0 && lo == 0, pair, part);
+            }
+        }
         __syncthreads();
     }
 
-    // ---- write the window back (positions >= t0 of every layer)
+    // ---- write the window back (16-byte stores from position s0 rounded down to 4)
     {
-        const int span = wlen - s0;
-        const int per = (M + 1) * ncb;
-        for (int e = tid; e < per * span; e += NT) {
-            const int s = s0 + e % span;
-            const int rest = e / span;
-            const int i = rest % ncb;
-            const int l = rest / ncb;
+        constexpr int PER = W / 4;
+        const int c4lo = s0 >> 2;
+        const int span = PER - c4lo;
+        const int total = (M + 1) * ncb * span;
+        for (int e = tid; e < total; e += NT) {
+            const int row = e / span, c4 = c4lo + (e - row * span);
+            const int l = row / ncb, i = row - l * ncb;
             const long long g = (long long)(i / nch) * D + c0 + (i % nch);
-            a.act[((long long)l * G + g) * L + kW + s] = slot[(l * CPB + i) * P + s];
+            const float* s = slot + (l * CPB + i) * P + 4 * c4;
+            *reinterpret_cast<float4*>(a.act + ((long long)l * G + g) * L + kW + 4 * c4) =
+                make_float4(s[0], s[1], s[2], s[3]);
         }
     }
 }

@@ -111,9 +111,11 @@ CASES_TF = [
     # M, B, D, L, W (None: library's choice)
     (3, 2, 5, 256, None),
     (2, 1, 3, 2048, 32),
-    (4, 3, 7, 1024, 16),
+    (4, 3, 7, 1024, 32),
     (1, 1, 16, 1024, 64),
     (2, 2, 33, 4096, 128),
+    (2, 1, 5, 4096, 256),
+    (18, 2, 3, 1024, 64),
 ]
 
 
@@ -201,7 +203,7 @@ def test_generate_continues_across_calls_and_reset_repeats(window):
 
 @pytest.mark.parametrize("force", ["direct", "fft"])
 def test_forced_tau_everywhere(force, window):
-    window(16)
+    window(32)
     M, B, D, L = 2, 1, 4, 1 << 13
     h = synth.filters(M, D, L, seed=4, decay=False)
     x = synth.inputs(L, B, D, seed=4)
