@@ -232,7 +232,13 @@ def main():
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1) / args.steps
     launches = ctx.info().launches - launches0
-    tr = ctx.trace() if trace else {}
+    tr, perq = ctx.trace(per_block_size=True) if trace else ({}, {})
+    classes_q = {}
+    for q in perq:
+        impl = info.tau[q]
+        name = ("block_direct" if impl == fi.FI_TAU_DIRECT else
+                ("block_split" if q > 14 else "block_fft"))
+        classes_q.setdefault(name, set()).add(q)
     if world > 1:
         tms = torch.tensor([ms], device="cuda")
         dist.all_reduce(tms, op=dist.ReduceOp.MAX)
@@ -273,23 +279,27 @@ def main():
 
     roof = None
     if tr:
+        # dominant kernel class by device time in the traced (last timed) step
         dom = max(tr, key=lambda k: tr[k][1])
         n_l, tot_us, max_us = tr[dom]
-        avg_s = tot_us / n_l * 1e-6
         if dom == "window":
             per_launch = window_bytes(M, B, D, L, info.window)
-            unit_desc = "W=%d tokens x (red cells + blocks of edge < W), %d layers x %d channels" % (
-                info.window, M, D)
+            work = per_launch * n_l
+            unit_desc = ("W=%d tokens x (red cells + blocks of edge < W) x %d layers x %d channels"
+                         % (info.window, M, D))
         else:
-            per_launch = byts / max(1, n_l)
-            unit_desc = "mean block launch"
-        ach = per_launch / avg_s / 1e9
+            # block launches: algorithmic bytes of each block size launched in this class
+            cls_q = {q: v for q, v in perq.items() if q in classes_q.get(dom, ())}
+            work = sum(v[0] * level_bytes(M, B, D, L, q) for q, v in cls_q.items())
+            per_launch = work / max(1, n_l)
+            unit_desc = "blocks of edge 2^q for q in %s, every layer and channel" % sorted(cls_q)
+        ach = work / (tot_us * 1e-6) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(ach / hbm, 4), "traffic": None, "kernel": dom,
                 "launches_per_step": n_l, "avg_launch_us": round(tot_us / n_l, 2),
-                "bytes_per_launch": per_launch, "per_launch_work": unit_desc,
-                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
-                else "fallback 6.65 TB/s"}
+                "bytes_per_launch": int(per_launch), "per_launch_work": unit_desc,
+                "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                                else "fallback 6.65 TB/s")}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -334,6 +344,7 @@ def main():
         "cpu_baseline": cpu,
         "clocks": clk,
         "kernel_time_us": {k: round(v[1], 1) for k, v in tr.items()},
+        "block_time_us": {str(q): round(v[1], 1) for q, v in sorted(perq.items())},
         "setup_s": {"filters": round(t_gen, 2), "create": round(t_create, 2)},
         "outputs_finite": finite,
         "context": "pages' figures (H100/A100, precision not stated): 110x mixer and 7.8x end-to-end "

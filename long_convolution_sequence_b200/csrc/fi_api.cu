@@ -210,8 +210,8 @@ size_t win_smem_bytes(int W, int M, int B, int kch) {
     return (size_t)((M + 1) * kch * B + M * kch) * (W + 2) * sizeof(float);
 }
 
-// chain registers of the window kernel are unrolled up to MAXM layers
-int win_maxm(int M) { return M <= 8 ? 8 : (M <= 20 ? 20 : (M <= 40 ? 40 : 0)); }
+// chain registers of the window kernel are unrolled up to MAXM layers (18: exact)
+int win_maxm(int M) { return M <= 8 ? 8 : (M == 18 ? 18 : (M <= 20 ? 20 : (M <= 40 ? 40 : 0))); }
 
 // ---------------------------------------------------------------- kernel launchers
 template <int LOGN>
@@ -288,7 +288,7 @@ int launch_spectra(int logn, const float* taps, long long ld, int count, int nsp
 
 template <int W, int MAXM>
 int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
-    k_window<W, MAXM><<<c->win_ncta, kWinThreads, c->win_smem, st>>>(a);
+    k_window<W, MAXM, MAXM == 18><<<c->win_ncta, kWinThreads, c->win_smem, st>>>(a);
     CK(cudaGetLastError());
     return FI_OK;
 }
@@ -297,6 +297,7 @@ template <int W>
 int launch_window_w(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
     switch (win_maxm(c->M)) {
         case 8: return launch_window_t<W, 8>(c, a, st);
+        case 18: return launch_window_t<W, 18>(c, a, st);
         case 20: return launch_window_t<W, 20>(c, a, st);
         case 40: return launch_window_t<W, 40>(c, a, st);
         default: return set_err(FI_EINVAL, "window kernel supports at most 40 layers");
@@ -326,9 +327,10 @@ int attr_fft() {
 
 template <int W>
 int attr_window() {
-    CK(cudaFuncSetAttribute(k_window<W, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<W, 20>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<W, 40>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 18, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 20, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 40, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
     return FI_OK;
 }
 
@@ -613,7 +615,7 @@ int choose_window(fi_ctx* c) {
     const int ncta = (c->D + kch - 1) / kch;
     const int per_sm = (ncta + c->nsm - 1) / c->nsm;
     if (!win_maxm(c->M)) return FI_OK;
-    const int cand[] = {256, 128, 64, 32};
+    const int cand[] = {128, 64, 256, 32};
     for (int W : cand) {
         if (forced && W != forced) continue;
         if (W > c->L) continue;

@@ -31,10 +31,16 @@ namespace fi {
 __host__ __device__ __forceinline__ long long lowbit(long long n) { return n & (-n); }
 __host__ __device__ __forceinline__ bool is_pow2(long long n) { return n > 0 && (n & (n - 1)) == 0; }
 
-// tanh(y) = 1 - 2 / (1 + 2^(2 y log2(e))), from the definition of tanh through the
-// exponential, evaluated with the SFU's base-2 exponential and reciprocal.  Absolute
-// error below 3e-7 over the reals (checked against fp64 tanh and CUDA's tanhf by
-// the GPU tests); saturates exactly to +-1 for large |y|.
+// tanh on the SFU, accurate in relative terms:
+//  * |y| >= 1/8: tanh(y) = 1 - 2 / (1 + 2^(K y)) with K = 2 / ln 2 (the definition of
+//    tanh through the exponential), evaluated with the SFU's base-2 exponential and
+//    reciprocal; absolute error ~2e-7, so relative error < 2e-6; saturates exactly
+//    to +-1 for large |y|;
+//  * |y| < 1/8: the odd Taylor series tanh(y) = y (1 - y^2/3 + 2 y^4/15 - 17 y^6/315),
+//    whose first omitted term (62/2835 y^9) is below 2e-9 relative there.
+// Both are computed and one is selected, so the latency is the exponential path's.
+constexpr float kTanhK = 2.8853900817779268f;      // 2 / ln 2
+constexpr float kTanhSmallZ = 0.36067376022224085f;  // K / 8: |y| < 1/8  <=>  |K y| < K / 8
 __device__ __forceinline__ float sfu_ex2(float x) {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -45,14 +51,22 @@ __device__ __forceinline__ float sfu_rcp(float x) {
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
+// odd series part for small arguments: y * (1 + x (-1/3 + x (2/15 - 17/315 x))), x = y^2
+__device__ __forceinline__ float tanh_series(float y) {
+    const float x = y * y;
+    float q = fmaf(x, -0.053968253968253971f, 0.13333333333333333f);
+    q = fmaf(x, q, -0.33333333333333331f);
+    q = fmaf(x, q, 1.0f);
+    return y * q;
+}
 __device__ __forceinline__ float act_tanh(float y) {
 #ifdef FI_TANH_LIBM
     return tanhf(y);
 #else
-    const float two_log2e = 2.8853900817779268f;  // 2 / ln 2
-    float e = sfu_ex2(two_log2e * y);
-    float r = sfu_rcp(1.0f + e);
-    return fmaf(-2.0f, r, 1.0f);
+    const float z = kTanhK * y;
+    const float r = sfu_rcp(1.0f + sfu_ex2(z));
+    const float big = fmaf(-2.0f, r, 1.0f);
+    return fabsf(z) < kTanhSmallZ ? tanh_series(y) : big;
 #endif
 }
 
@@ -527,61 +541,101 @@ __device__ __forceinline__ int cover_range(int T, int s0, int hi, int* top) {
     return lo;
 }
 
-// sum over j = jb, jb+2, ... < je of in[j] * tp[T - j]
-__device__ __forceinline__ float dot_stride2(const float* in, const float* tp, int T, int jb, int je) {
+// One lane of a helper pair: sum over j = lo + part + 2k (k < n2) of in[j] * tp[T - j],
+// where n2 = ceil((hi - lo + 1) / 2) is the same for both lanes, so the two lanes run
+// identical trip counts (no divergence); the odd lane's last term, which would fall
+// one past hi when the range length is odd, is masked.
+__device__ __forceinline__ float dot_pair(const float* in, const float* tp, int T, int lo, int hi, int part) {
+    const int n2 = (hi - lo + 2) >> 1;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int j = jb;
-    for (; j + 6 < je; j += 8) {
+    int k = 0;
+    const int jb = lo + part;
+    for (; k + 4 < n2; k += 4) {  // k .. k+3 < n2 - 1: in range for both lanes
+        const int j = jb + 2 * k;
         a0 = fmaf(in[j], tp[T - j], a0);
         a1 = fmaf(in[j + 2], tp[T - j - 2], a1);
         a2 = fmaf(in[j + 4], tp[T - j - 4], a2);
         a3 = fmaf(in[j + 6], tp[T - j - 6], a3);
     }
-    for (; j < je; j += 2) a0 = fmaf(in[j], tp[T - j], a0);
+    for (; k < n2; ++k) {
+        const int j = jb + 2 * k;
+        const bool ok = j <= hi;
+        const int jc = ok ? j : hi;
+        a0 = fmaf(ok ? in[jc] : 0.f, tp[T - jc], a0);
+    }
     return (a0 + a1) + (a2 + a3);
+}
+
+// One helper pair's first (layer, chain) item: shared-memory offsets of its input
+// row, tap row and output row (out < 0: none).  Shapes with more items than pairs
+// hand the pair further items pair + k * kWinPairs, decoded on the fly.
+struct PairItem {
+    int in, tp, out;
+};
+
+struct ItemGeom {
+    int nitems, ncb, nch, CPB, kch, P, tap0;
+};
+
+__device__ __forceinline__ PairItem decode_item(const ItemGeom& g, int it) {
+    PairItem r;
+    if (it < g.nitems) {
+        const int l = it / g.ncb + 1, i = it - (l - 1) * g.ncb;
+        r.in = ((l - 1) * g.CPB + i) * g.P;
+        r.tp = g.tap0 + ((l - 1) * g.kch + (i % g.nch)) * g.P;
+        r.out = (l * g.CPB + i) * g.P;
+    } else {
+        r.in = r.tp = 0;
+        r.out = -1;
+    }
+    return r;
+}
+
+__device__ __forceinline__ void add_row(float* sm, const PairItem& it, int T, int lo, int hi, bool ow, int part) {
+    const bool mine = it.out >= 0;
+    float acc = mine ? dot_pair(sm + it.in, sm + it.tp, T, lo, hi, part) : 0.f;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if (part == 0 && mine) {
+        float* o = sm + it.out + T;
+        *o = ow ? acc : *o + acc;
+    }
 }
 
 // Helper pairs add the rows over inputs [lo, hi] onto position T of every
 // (layer, chain); overwrite when these rows include the position's first writer.
-template <int P>
-__device__ __forceinline__ void helper_rows(float* slot, const float* tap, int M, int ncb, int nch, int CPB,
-                                            int kch, int T, int lo, int hi, bool ow, int pair, int part) {
-    const int items = M * ncb;
-    for (int base = 0; base < items; base += kWinPairs) {
-        const int it = base + pair;
-        float acc = 0.f;
-        int l = 0, i = 0;
-        if (it < items) {
-            l = it / ncb + 1;
-            i = it - (l - 1) * ncb;
-            const float* in = slot + ((l - 1) * CPB + i) * P;
-            const float* tp = tap + ((l - 1) * kch + (i % nch)) * P;
-            acc = dot_stride2(in, tp, T, lo + part, hi + 1);
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        if (it < items && part == 0) {
-            float* o = slot + (l * CPB + i) * P + T;
-            *o = ow ? acc : *o + acc;
-        }
-    }
+// All lanes of a (fully active) helper warp make the same shuffles: the extra-item
+// loop runs to the warp's largest count and lanes past their own count add 0.
+__device__ __noinline__ void helper_rows_more(float* sm, const ItemGeom& g, int pair, int T, int lo, int hi,
+                                              bool ow, int part) {
+    const int mine_n = pair < g.nitems ? (g.nitems - pair + kWinPairs - 1) / kWinPairs : 0;
+    const int nwarp = (int)__reduce_max_sync(0xffffffffu, (unsigned)mine_n);
+    for (int k = 1; k < nwarp; ++k) add_row(sm, decode_item(g, pair + k * kWinPairs), T, lo, hi, ow, part);
 }
 
-template <int W, int MAXM>
+__device__ __forceinline__ void helper_rows(float* sm, const ItemGeom& g, const PairItem& first, bool more,
+                                            int pair, int T, int lo, int hi, bool ow, int part) {
+    add_row(sm, first, T, lo, hi, ow, part);
+    if (more) helper_rows_more(sm, g, pair, T, lo, hi, ow, part);
+}
+
+template <int W, int MAXM, bool EXACT>
 __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     extern __shared__ float4 sm4[];
     float* sm = reinterpret_cast<float*>(sm4);
     constexpr int NT = kWinThreads;
     constexpr int P = W + 2;  // row pitch: the two lanes of a helper pair and consecutive rows hit distinct banks
-    constexpr float K = 2.8853900817779268f;  // 2 / ln 2: tanh(y) = 1 - 2 / (1 + 2^(K y))
-    const int M = a.M, B = a.B, D = a.D, kch = a.kch;
+    constexpr float K = kTanhK;
+    const int M = EXACT ? MAXM : a.M;
+    const int B = a.B, D = a.D, kch = a.kch;
     const long long L = a.L, G = a.G;
     const int c0 = blockIdx.x * kch;
     const int nch = min(kch, D - c0);
     const int ncb = nch * B;
     const int CPB = kch * B;
-    float* slot = sm;                                   // [(M+1) * CPB][P]
-    float* tap = sm + (size_t)(M + 1) * CPB * P;         // [M * kch][P]
-    const long long kW = (a.t0 / W) * (long long)W;      // windows never cross L (W divides L)
+    const int tap0 = (M + 1) * CPB * P;
+    float* slot = sm;               // [(M+1) * CPB][P]
+    float* tap = sm + tap0;         // [M * kch][P]
+    const long long kW = (a.t0 / W) * (long long)W;  // windows never cross L (W divides L)
     const int s0 = (int)(a.t0 - kW), s1 = (int)(a.t1 - kW);
     const int tid = threadIdx.x;
 
@@ -609,7 +663,7 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                         const int r2 = row - rows_slot;
                         const int l = r2 / nch, ci = r2 - l * nch;
                         src = a.h + ((long long)l * D + c0 + ci) * L + 4 * c4;
-                        dst[u] = (M + 1) * CPB * P + (l * kch + ci) * P + 4 * c4;
+                        dst[u] = tap0 + (l * kch + ci) * P + 4 * c4;
                     }
                     v[u] = __ldg(reinterpret_cast<const float4*>(src));
                 }
@@ -643,58 +697,88 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
         __syncthreads();
     }
 
-    // ---- tokens
+    // ---- per-launch setup: chain constants in registers, helper item lists
     const int lane = tid;
     const bool chain = tid < 32 && lane < ncb;
     long long gch = 0;
     int cich = 0;
+    float hs[MAXM], m2hs[MAXM], kh1[MAXM], aprev[MAXM + 1];
     if (chain) {
         cich = lane % nch;
         gch = (long long)(lane / nch) * D + c0 + cich;
+#pragma unroll
+        for (int l = 1; l <= MAXM; ++l) {
+            const int lc = l <= M ? l : M;
+            const float* tl = tap + ((lc - 1) * kch + cich) * P;
+            hs[l - 1] = K * tl[0];
+            m2hs[l - 1] = -2.f * K * tl[0];
+            kh1[l - 1] = K * tl[1];
+        }
+        // activations of token t0-1 (used only from the second step on)
+#pragma unroll
+        for (int l = 0; l <= MAXM; ++l) aprev[l] = 0.f;
     }
     const int pair = (tid - 32) >> 1, part = tid & 1;
+    ItemGeom geom;
+    geom.nitems = M * ncb;
+    geom.ncb = ncb;
+    geom.nch = nch;
+    geom.CPB = CPB;
+    geom.kch = kch;
+    geom.P = P;
+    geom.tap0 = tap0;
+    const PairItem first = decode_item(geom, tid >= 32 ? pair : geom.nitems);
+    const bool more = geom.nitems > kWinPairs;  // uniform over the CTA
+
+    // ---- tokens
     for (int s = s0; s < s1; ++s) {
         const long long t = kW + s;
         if (tid < 32) {
             if (chain) {
                 // running sums of every layer first (independent of the chain), then the
-                // link chain in registers: z_l = K y_l, r_l = 1 / (1 + 2^z_l), a_l = 1 - 2 r_l,
-                // z_{l+1} = (-2 K h0) r_l + (K h0 + K p_{l+1})
-                const bool newest = s > s0;
-                float c1[MAXM], c2[MAXM];
+                // link chain in registers on z_l = K y_l:  r = 1 / (1 + 2^z), a_l = 1 - 2r
+                // (or the series for small |y|), z_{l+1} = K h0 a_l + K p_{l+1}, with the
+                // large-|y| form of z_{l+1} folded as (-2 K h0) r + (K h0 + K p_{l+1}).
+                float p[MAXM];
 #pragma unroll
                 for (int l = 1; l <= MAXM; ++l) {
-                    if (l <= M) {
-                        const float* tl = tap + ((l - 1) * kch + cich) * P;
-                        float p = (t == 0) ? 0.f : slot[(l * CPB + lane) * P + s];
-                        if (newest) p = fmaf(tl[1], slot[((l - 1) * CPB + lane) * P + s - 1], p);
-                        const float hs = K * tl[0];
-                        if (l == 1) {
-                            c1[0] = hs;
-                            c2[0] = K * p;
-                        } else {
-                            c1[l - 1] = -2.f * hs;
-                            c2[l - 1] = fmaf(K, p, hs);
+                    const int lc = l <= M ? l : M;
+                    p[l - 1] = slot[(lc * CPB + lane) * P + s];
+                }
+                const float a0 = slot[lane * P + s];
+                const bool newest = s > s0;  // row 0 of block n = t still lacks a^{l-1}_{t-1}
+                const bool zero = t == 0;    // position 0 has no block: its running sum is 0
+                float kp[MAXM], hsc[MAXM];
+#pragma unroll
+                for (int l = 1; l <= MAXM; ++l) {
+                    float v = zero ? 0.f : K * p[l - 1];
+                    if (newest) v = fmaf(kh1[l - 1], aprev[l - 1], v);
+                    kp[l - 1] = v;
+                    hsc[l - 1] = hs[l - 1] + v;
+                }
+                aprev[0] = a0;
+                float z = fmaf(hs[0], a0, kp[0]);
+                float av = 0.f;
+#pragma unroll
+                for (int l = 1; l <= MAXM; ++l) {
+                    if (EXACT || l <= M) {
+                        const float r = sfu_rcp(1.0f + sfu_ex2(z));
+                        const bool small = fabsf(z) < kTanhSmallZ;
+                        const float as = tanh_series(z * (1.0f / K));
+                        av = small ? as : fmaf(-2.f, r, 1.f);
+                        slot[(l * CPB + lane) * P + s] = av;
+                        aprev[l] = av;
+                        if (l < MAXM && (EXACT || l < M)) {
+                            const float zl = small ? fmaf(hs[l], as, kp[l]) : fmaf(m2hs[l], r, hsc[l]);
+                            z = zl;
                         }
                     }
                 }
-                const float a0 = slot[lane * P + s];
-                float z = fmaf(c1[0], a0, c2[0]);
-                float r = sfu_rcp(1.0f + sfu_ex2(z));
-                slot[(CPB + lane) * P + s] = fmaf(-2.f, r, 1.f);
-#pragma unroll
-                for (int l = 2; l <= MAXM; ++l) {
-                    if (l <= M) {
-                        z = fmaf(c1[l - 1], r, c2[l - 1]);
-                        r = sfu_rcp(1.0f + sfu_ex2(z));
-                        slot[(l * CPB + lane) * P + s] = fmaf(-2.f, r, 1.f);
-                    }
-                }
+                // z now holds K y^M (the last layer's link does not advance it)
                 a.out[(t - a.tx) * G + gch] = z * (1.0f / K);
                 if (a.closed) {
-                    const float aM = fmaf(-2.f, r, 1.f);
-                    if (s + 1 < W) slot[lane * P + s + 1] = aM;
-                    else if (t + 1 < L) a.act[gch * L + t + 1] = aM;
+                    if (s + 1 < W) slot[lane * P + s + 1] = av;
+                    else if (t + 1 < L) a.act[gch * L + t + 1] = av;
                 }
             }
         } else {
@@ -702,7 +786,7 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             if (T < W) {
                 int top;
                 const int lo = cover_range(T, s0, T, &top);
-                helper_rows<P>(slot, tap, M, ncb, nch, CPB, kch, T, lo, s - 1, kW == 0 && lo == 0, pair, part);
+                helper_rows(sm, geom, first, more, pair, T, lo, s - 1, kW == 0 && lo == 0, part);
             }
         }
         __syncthreads();
@@ -721,26 +805,37 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             for (int T = s1 + 1; T < W; ++T) {
                 int top;
                 const int lo = cover_range(T, s0, s1, &top);
-                if (lo >= 0)
-                    helper_rows<P>(slot, tap, M, ncb, nch, CPB, kch, T, lo, top, kW == 0 && lo == 0, pair, part);
+                if (lo >= 0) helper_rows(sm, geom, first, more, pair, T, lo, top, kW == 0 && lo == 0, part);
             }
         }
         __syncthreads();
     }
 
-    // ---- write the window back (16-byte stores from position s0 rounded down to 4)
+    // ---- write the window back (16-byte stores from position s0 rounded down to 4);
+    // thread -> (column group, first row), rows advance by a fixed stride
     {
         constexpr int PER = W / 4;
         const int c4lo = s0 >> 2;
         const int span = PER - c4lo;
-        const int total = (M + 1) * ncb * span;
-        for (int e = tid; e < total; e += NT) {
-            const int row = e / span, c4 = c4lo + (e - row * span);
-            const int l = row / ncb, i = row - l * ncb;
-            const long long g = (long long)(i / nch) * D + c0 + (i % nch);
-            const float* s = slot + (l * CPB + i) * P + 4 * c4;
-            *reinterpret_cast<float4*>(a.act + ((long long)l * G + g) * L + kW + 4 * c4) =
-                make_float4(s[0], s[1], s[2], s[3]);
+        const int rows = (M + 1) * ncb;
+        const int rstride = NT / span;  // span <= W/4 <= 64 < NT
+        const int c4 = c4lo + tid % span;
+        int row = tid / span;
+        if (row < rstride) {
+            int l = row / ncb, i = row - l * ncb;
+            const int dl = rstride / ncb, di = rstride - dl * ncb;
+            for (; row < rows; row += rstride) {
+                const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+                const float* sp = slot + (l * CPB + i) * P + 4 * c4;
+                *reinterpret_cast<float4*>(a.act + ((long long)l * G + g) * L + kW + 4 * c4) =
+                    make_float4(sp[0], sp[1], sp[2], sp[3]);
+                l += dl;
+                i += di;
+                if (i >= ncb) {
+                    i -= ncb;
+                    ++l;
+                }
+            }
         }
     }
 }

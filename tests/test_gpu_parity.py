@@ -78,20 +78,29 @@ def test_tau_fft_matches_oracle(U):
 
 # ------------------------------------------------------------------ block function
 def test_tanh_of_the_red_cell_is_accurate():
-    # one layer, h = delta_0: a^1_0 = tanh(x_0) for a sweep of x_0 values
-    D = 8192
-    h = np.zeros((1, D, 2), np.float32)
-    h[0, :, 0] = 1.0
-    x = np.linspace(-12, 12, D, dtype=np.float32).reshape(1, 1, D)
-    with fi.FlashInference(1, 1, D, 2, h) as ctx:
-        y = np.empty((1, 1, D), np.float32)
-        ctx.forward(x, 1, y)
-        a = np.empty((1, 1, D), np.float32)
-        ctx.read_layer(1, 0, 1, a)
-    np.testing.assert_array_equal(y, x)
-    err = np.abs(a.astype(np.float64) - np.tanh(x.astype(np.float64)))
-    assert err.max() < 5e-7
-    assert a[0, 0, 0] == -1.0 and a[0, 0, -1] == 1.0
+    # one layer, h = delta_0: a^1_0 = tanh(x_0) for a sweep of x_0 values, on both the
+    # per-token and the window path; absolute and relative accuracy
+    grid = np.linspace(-12, 12, 4096)
+    tiny = np.logspace(-30, 0, 2048)
+    x = np.concatenate([grid, tiny, -tiny]).astype(np.float32)
+    D = x.size
+    for L in (2, 64):
+        h = np.zeros((1, D, L), np.float32)
+        h[0, :, 0] = 1.0
+        with fi.FlashInference(1, 1, D, L, h) as ctx:
+            xs = np.zeros((L, 1, D), np.float32)
+            xs[0, 0] = x
+            y = np.empty((L, 1, D), np.float32)
+            ctx.forward(xs, L, y)
+            a = np.empty((1, 1, D), np.float32)
+            ctx.read_layer(1, 0, 1, a)
+        np.testing.assert_allclose(y[0, 0], x, rtol=3e-7, atol=0)  # window path returns (K y) / K
+        ref = np.tanh(x.astype(np.float64))
+        got = a[0, 0].astype(np.float64)
+        assert np.abs(got - ref).max() < 5e-7
+        nz = np.abs(ref) > 1e-30
+        assert (np.abs(got - ref)[nz] / np.abs(ref[nz])).max() < 3e-6
+        assert got[np.argmin(x)] == -1.0 and got[np.argmax(x)] == 1.0
 
 
 # ------------------------------------------------------------------ schedule
@@ -116,6 +125,8 @@ CASES_TF = [
     (2, 2, 33, 4096, 128),
     (2, 1, 5, 4096, 256),
     (18, 2, 3, 1024, 64),
+    (36, 1, 2, 512, 64),
+    (20, 1, 3, 512, 128),
 ]
 
 
