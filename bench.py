@@ -35,6 +35,9 @@ WORKLOADS = {
     "headline": (18, 1, 864, 1 << 17),
     "hyena_shape": (18, 4, 768, 1 << 15),
     "tiny": (1, 1, 16, 1 << 10),
+    # the headline stack at a shorter length: a few GB on the device, every launch
+    # still larger than L2 (used for profiler captures)
+    "short": (18, 1, 864, 1 << 14),
 }
 FALLBACK_HBM_GBS = 6650.0
 FP32_LANES_PER_SM = 128
@@ -156,6 +159,28 @@ def oracle_sample_size(M, L, budget_s=15.0, rate=1.0e9):
     return min(T_s, L)
 
 
+# ------------------------------------------------------------------ ranks
+def rank_seed(rank):
+    """Seed of rank r's start token: every replica generates its own sequence."""
+    return rank
+
+
+def max_over_ranks(x, world, device):
+    """The largest of the ranks' values (every rank gets it); the identity at N=1."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, B, L, ms_max):
+    """Whole-job throughput: the tokens all ranks generated over the slowest rank's time."""
+    return world * B * L / (ms_max / 1000.0)
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -192,7 +217,7 @@ def main():
 
     t_setup = time.perf_counter()
     h = synth.filters(M, D, L, seed=0)
-    x0 = synth.start_token(B, D, seed=rank)
+    x0 = synth.start_token(B, D, seed=rank_seed(rank))
     t_gen = time.perf_counter() - t_setup
     t0 = time.perf_counter()
     ctx = fi.FlashInference(M, B, D, L, h)
@@ -239,10 +264,7 @@ def main():
         name = ("block_direct" if impl == fi.FI_TAU_DIRECT else
                 ("block_split" if q > 14 else "block_fft"))
         classes_q.setdefault(name, set()).add(q)
-    if world > 1:
-        tms = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
-        ms = float(tms.item())
+    ms = max_over_ranks(ms, world, "cuda")
 
     # end to end through the public API: host (pinned) start token in, host result out
     x0_h = torch.from_numpy(x0).pin_memory()
@@ -257,10 +279,7 @@ def main():
         ctx.reset()
         ctx.generate(x0_h, L, out_h)
     e2e_sec = (time.perf_counter() - t0) / e2e_steps
-    if world > 1:
-        te = torch.tensor([e2e_sec], device="cuda")
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_sec = float(te.item())
+    e2e_sec = max_over_ranks(e2e_sec, world, "cuda")
     finite = bool(np.isfinite(out_h.numpy()).all())
 
     if rank != 0:
@@ -272,7 +291,7 @@ def main():
 
     hbm, peak_kind, sm_mhz = peaks()
     tokens = world * B * L
-    value = tokens / (ms / 1000.0)
+    value = job_tokens_per_s(world, B, L, ms)
     byts, flops = model_bytes_flops(M, B, D, L)
     fp32_peak = info.sm_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6
     t_roof = max(byts / (hbm * 1e9), flops / fp32_peak)
