@@ -180,6 +180,28 @@ int fi_debug_schedule(const fi_ctx *ctx, int n, int *U, int *impl, int *src_lo,
 int fi_tau(int impl, int U, int count, const float *blocks, const float *taps, int ldt,
            float *out, int accumulate);
 
+/* The FFT tau of fi_tau (impl = FI_TAU_FFT) for callers that must not allocate
+ * device memory.  The paper has no counterpart: this entry point exists for
+ * callers whose device memory is owned by someone else -- an application whose
+ * pool allocator has reserved the GPU's memory up front (so cudaMalloc fails or
+ * fragments that pool), or a loop that cannot afford the device-wide
+ * synchronisation cudaMalloc and cudaFree may imply.
+ * Arguments and result are those of fi_tau with impl = FI_TAU_FFT: count blocks of
+ * edge U (8 <= U <= 65536, a power of two), taps rows of ldt >= 2U (even) floats,
+ * out[i][r] (+)= tau; all pointers DEVICE memory, 8-byte aligned; the caller owns
+ * them.  Every temporary (twiddle table, filter spectra, sub-block spectra) lives
+ * in one fixed 8 MiB array in device memory, part of the library image, which every
+ * GPU that loads the library holds until the process exits; large counts are
+ * processed in chunks that fit it.  The first call on a device sets that device up
+ * (looks up the array's device address and writes the twiddle table with a
+ * synchronous copy), so make it before any stream capture.  Nothing in the array
+ * needs to start at zero: each call writes every part it reads.  All calls share
+ * the array, so calls that overlap on the GPU race (for example from two host
+ * threads); calls are serialised on the legacy default stream and return after
+ * completion.  FI_EINVAL for U beyond 65536 (or any fi_tau argument error). */
+int fi_tau_fft_noalloc(int U, int count, const float *blocks, const float *taps, int ldt,
+                       float *out, int accumulate);
+
 /* Message of the last failure on the calling thread ("" if none). */
 const char *fi_last_error(void);
 

@@ -62,6 +62,7 @@ SIGNATURES = {
     "fi_trace_read": (_I, [_P, ctypes.POINTER(fi_trace)]),
     "fi_debug_schedule": (_I, [_P, _I] + [ctypes.POINTER(_I)] * 5),
     "fi_tau": (_I, [_I, _I, _I, _P, _P, _I, _P, _I]),
+    "fi_tau_fft_noalloc": (_I, [_I, _I, _P, _P, _I, _P, _I]),
     "fi_last_error": (ctypes.c_char_p, []),
     "fi_version": (ctypes.c_char_p, []),
 }
@@ -200,3 +201,12 @@ def tau(impl: int, U: int, blocks, taps, out, accumulate: bool = False):
     count = blocks.shape[0]
     ldt = taps.shape[1]
     _check(get_lib().fi_tau(impl, U, count, _ptr(blocks), _ptr(taps), ldt, _ptr(out), int(bool(accumulate))))
+
+
+def tau_fft_noalloc(U: int, blocks, taps, out, accumulate: bool = False):
+    """FFT tau without device allocations (fixed library scratch): see
+    fi_tau_fft_noalloc in fi.h."""
+    count = blocks.shape[0]
+    ldt = taps.shape[1]
+    _check(get_lib().fi_tau_fft_noalloc(U, count, _ptr(blocks), _ptr(taps), ldt, _ptr(out),
+                                        int(bool(accumulate))))

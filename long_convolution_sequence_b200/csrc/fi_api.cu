@@ -29,6 +29,12 @@
 
 using namespace fi;
 
+// Fixed device scratch of fi_tau_fft_noalloc (8 MiB, in every device that loads the
+// library, until the process exits).  Host code must not use the symbol as a device
+// address: the address comes from cudaGetSymbolAddress at set-up.
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 thread_local char g_err[1024] = "";
@@ -442,6 +448,108 @@ int tau_impl(fi_ctx* tmp, int impl, int U, int q, int count, const float* blocks
         }
     }
     if (rc) return rc;
+    CK(cudaStreamSynchronize(st));
+    return FI_OK;
+}
+
+// ---------------------------------------------------------------- allocation-free FFT tau
+// Scratch of fi_tau_fft_noalloc: one fixed array per device, part of the library's
+// device image, so it exists from module load to process exit and needs no
+// cudaMalloc.  Layout (complex64 entries): [0, 2^kTwLog) twiddles, written once per
+// device at set-up; then the filter spectra of one chunk of items; then, for block
+// sizes above one CTA's FFT, the split kernel's per-CTA sub-block spectra.
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float2* g_noalloc_base[kNoAllocMaxDevices] = {};
+
+// Once per device, with that device current: resolve the array's device address
+// (the host-side symbol is only a stand-in) and store the twiddle table in it.
+int noalloc_setup(int dev, float2** base) {
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return set_err(FI_EINVAL, "fi_tau_fft_noalloc: device ordinal %d above %d", dev, kNoAllocMaxDevices - 1);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_base[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();
+            return set_err(FI_ECUDA, "fi_tau_fft_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+        }
+        const int nt = 1 << kTwLog;
+        std::vector<float2> tw(nt);
+        for (int k = 0; k < nt; ++k) {
+            const double ang = -2.0 * M_PI * (double)k / (double)nt;
+            tw[k] = make_float2((float)cos(ang), (float)sin(ang));
+        }
+        e = cudaMemcpy(p, tw.data(), sizeof(float2) * nt, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return set_err(FI_ECUDA, "fi_tau_fft_noalloc: twiddle upload failed: %s", cudaGetErrorString(e));
+        }
+        g_noalloc_base[dev] = (float2*)p;
+    }
+    *base = g_noalloc_base[dev];
+    return FI_OK;
+}
+
+// The FFT tau of fi_tau, with every temporary carved out of the fixed array and the
+// items processed in chunks small enough to fit it.
+int tau_fft_noalloc_impl(int U, int q, int count, const float* blocks, const float* taps, int ldt, float* out,
+                         int accumulate) {
+    int dev = 0, nsm = 0;
+    CK(cudaGetDevice(&dev));
+    CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    float2* base = nullptr;
+    int rc = noalloc_setup(dev, &base);
+    if (rc) return rc;
+    const long long ntw = 1LL << kTwLog;
+    float2* spec = base + ntw;
+    const long long avail = (long long)(kNoAllocScratchBytes / sizeof(float2)) - ntw;
+    cudaStream_t st = nullptr;
+    TileArgs a;
+    memset(&a, 0, sizeof(a));
+    a.flat = 1;
+    a.ldt = ldt;
+    a.U = U;
+    a.overwrite = accumulate ? 0 : 1;
+    a.tw = base;
+    a.twlog = kTwLog;
+    if (q <= kLogSMax) {
+        const long long per_item = U + 1;
+        const int chunk = (int)std::min<long long>(count, avail / per_item);
+        for (int i0 = 0; i0 < count; i0 += chunk) {
+            const int n = std::min(chunk, count - i0);
+            const float* tp = taps + (long long)i0 * ldt;
+            if ((rc = launch_spectra(q, tp, ldt, n, 1, 0, spec, base, st))) return rc;
+            a.fin = blocks + (long long)i0 * U;
+            a.fout = out + (long long)i0 * U;
+            a.ftaps = tp;
+            a.count = n;
+            a.spec = spec;
+            a.spec_stride = per_item;
+            if ((rc = launch_fft_tile(q, a, st))) return rc;
+        }
+    } else {
+        const long long S = 1LL << kLogSMax;
+        const int nsub = (int)(U / S), nspec = 2 * nsub - 1;
+        const long long per_item = (long long)nspec * (S + 1), per_cta = (long long)nsub * (S + 1);
+        const int chunk = (int)std::min<long long>(std::min(count, nsm), avail / (per_item + per_cta));
+        float2* scr = spec + (long long)chunk * per_item;
+        for (int i0 = 0; i0 < count; i0 += chunk) {
+            const int n = std::min(chunk, count - i0);
+            const float* tp = taps + (long long)i0 * ldt;
+            if ((rc = launch_spectra(kLogSMax, tp, ldt, n, nspec, S, spec, base, st))) return rc;
+            a.fin = blocks + (long long)i0 * U;
+            a.fout = out + (long long)i0 * U;
+            a.ftaps = tp;
+            a.count = n;
+            a.spec = spec;
+            a.spec_stride = per_item;
+            a.nsub = nsub;
+            a.scratch = scr;
+            if ((rc = launch_split_tile(a, n, st))) return rc;
+        }
+    }
     CK(cudaStreamSynchronize(st));
     return FI_OK;
 }
@@ -1009,6 +1117,21 @@ int fi_tau(int impl, int U, int count, const float* blocks, const float* taps, i
     cudaFree(tmp.scratch);
     tmp.magic = 0;
     return rc;
+}
+
+int fi_tau_fft_noalloc(int U, int count, const float* blocks, const float* taps, int ldt, float* out,
+                       int accumulate) {
+    if (U < 1 || (U & (U - 1)) || count < 1 || !blocks || !taps || !out || ldt < 2 * U || (ldt & 1))
+        return set_err(FI_EINVAL, "fi_tau_fft_noalloc: need U a power of two, count >= 1, ldt >= 2U and even, "
+                                  "non-NULL pointers");
+    const int q = ctz64(U);
+    if (q < kFftQMin || q > kLogSMax + 2)
+        return set_err(FI_EINVAL, "fi_tau_fft_noalloc: U = %d outside [%d, %d], the largest block its fixed "
+                                  "%zu-byte scratch serves", U, 1 << kFftQMin, 1 << (kLogSMax + 2),
+                       kNoAllocScratchBytes);
+    int rc = set_all_attrs();
+    if (rc) return rc;
+    return tau_fft_noalloc_impl(U, q, count, blocks, taps, ldt, out, accumulate);
 }
 
 }  // extern "C"
