@@ -222,9 +222,9 @@ int win_maxm(int M) { return M <= 8 ? 8 : (M == 18 ? 18 : (M <= 20 ? 20 : (M <= 
 // ---------------------------------------------------------------- kernel launchers
 template <int LOGN>
 int launch_fft_tile_t(const TileArgs& a, cudaStream_t st) {
-    constexpr int NT = (1 << LOGN) / 4 < 32 ? 32 : ((1 << LOGN) / 4 > 1024 ? 1024 : (1 << LOGN) / 4);
-    const size_t smem = sizeof(float2) << LOGN;
-    k_tile_fft<LOGN, NT><<<a.count, NT, smem, st>>>(a);
+    using G = FftTile<LOGN>;
+    const int grid = (a.count + G::TPC - 1) / G::TPC;
+    k_block_fft<LOGN, kTwLog><<<grid, G::NT, G::smem, st>>>(a);
     CK(cudaGetLastError());
     return FI_OK;
 }
@@ -262,32 +262,38 @@ int launch_direct_tile(const TileArgs& a, cudaStream_t st) {
     return FI_OK;
 }
 
+// Spectra for the fused FFT tile kernel carry its 1/(2U) scale (fused_scale); the
+// split kernel's sub-block spectra are unscaled.
+float fused_scale(int q) { return 1.0f / (2.0f * (float)(1LL << q)); }
+// Complex entries per (layer, channel) spectrum of the fused kernel: bins 0..U plus
+// one pad entry, so that every spectrum starts on a 16-byte boundary (async copies).
+long long fused_stride(long long U) { return U + 2; }
+
 template <int LOGN>
 int launch_spectra_t(const float* taps, long long ld, int count, int nspec, long long offstep,
-                     float2* spec, const float2* tw, cudaStream_t st) {
+                     float2* spec, const float2* tw, cudaStream_t st, float scale, long long hstride) {
     constexpr int NT = (1 << LOGN) / 4 < 32 ? 32 : ((1 << LOGN) / 4 > 1024 ? 1024 : (1 << LOGN) / 4);
     const size_t smem = sizeof(float2) << LOGN;
-    // one CTA per (item, offset); chunk the grid to stay below 2^31 CTAs
-    k_spectra<LOGN, NT><<<count * nspec, NT, smem, st>>>(taps, ld, nspec, offstep, spec, tw, kTwLog);
+    k_spectra<LOGN, NT><<<count * nspec, NT, smem, st>>>(taps, ld, nspec, offstep, spec, tw, kTwLog, scale, hstride);
     CK(cudaGetLastError());
     return FI_OK;
 }
 
 int launch_spectra(int logn, const float* taps, long long ld, int count, int nspec, long long offstep,
-                   float2* spec, const float2* tw, cudaStream_t st) {
+                   float2* spec, const float2* tw, cudaStream_t st, float scale, long long hstride) {
     switch (logn) {
-        case 3: return launch_spectra_t<3>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 4: return launch_spectra_t<4>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 5: return launch_spectra_t<5>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 6: return launch_spectra_t<6>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 7: return launch_spectra_t<7>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 8: return launch_spectra_t<8>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 9: return launch_spectra_t<9>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 10: return launch_spectra_t<10>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 11: return launch_spectra_t<11>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 12: return launch_spectra_t<12>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 13: return launch_spectra_t<13>(taps, ld, count, nspec, offstep, spec, tw, st);
-        case 14: return launch_spectra_t<14>(taps, ld, count, nspec, offstep, spec, tw, st);
+        case 3: return launch_spectra_t<3>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 4: return launch_spectra_t<4>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 5: return launch_spectra_t<5>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 6: return launch_spectra_t<6>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 7: return launch_spectra_t<7>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 8: return launch_spectra_t<8>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 9: return launch_spectra_t<9>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 10: return launch_spectra_t<10>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 11: return launch_spectra_t<11>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 12: return launch_spectra_t<12>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 13: return launch_spectra_t<13>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
+        case 14: return launch_spectra_t<14>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
         default: return set_err(FI_EINVAL, "no spectrum kernel for 2^%d points", logn);
     }
 }
@@ -326,7 +332,8 @@ template <int LOGN>
 int attr_fft() {
     constexpr int NT = (1 << LOGN) / 4 < 32 ? 32 : ((1 << LOGN) / 4 > 1024 ? 1024 : (1 << LOGN) / 4);
     const int smem = (int)(sizeof(float2) << LOGN);
-    CK(cudaFuncSetAttribute(k_tile_fft<LOGN, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    CK(cudaFuncSetAttribute(k_block_fft<LOGN, kTwLog>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)FftTile<LOGN>::smem));
     CK(cudaFuncSetAttribute(k_spectra<LOGN, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     return FI_OK;
 }
@@ -426,10 +433,10 @@ int tau_impl(fi_ctx* tmp, int impl, int U, int q, int count, const float* blocks
         a.tw = tmp->tw;
         a.twlog = kTwLog;
         if (q <= kLogSMax) {
-            if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * (U + 1)))) return rc;
-            if ((rc = launch_spectra(q, taps, ldt, count, 1, 0, tmp->spec[0], tmp->tw, st))) return rc;
+            if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * fused_stride(U)))) return rc;
+            if ((rc = launch_spectra(q, taps, ldt, count, 1, 0, tmp->spec[0], tmp->tw, st, fused_scale(q), fused_stride(1LL << q)))) return rc;
             a.spec = tmp->spec[0];
-            a.spec_stride = U + 1;
+            a.spec_stride = fused_stride(U);
             rc = launch_fft_tile(q, a, st);
         } else {
             const long long S = 1LL << kLogSMax;
@@ -438,7 +445,7 @@ int tau_impl(fi_ctx* tmp, int impl, int U, int q, int count, const float* blocks
             CK(cudaGetDevice(&dev));
             CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
             if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * nspec * (S + 1)))) return rc;
-            if ((rc = launch_spectra(kLogSMax, taps, ldt, count, nspec, S, tmp->spec[0], tmp->tw, st))) return rc;
+            if ((rc = launch_spectra(kLogSMax, taps, ldt, count, nspec, S, tmp->spec[0], tmp->tw, st, 1.0f, S + 1))) return rc;
             if ((rc = dev_alloc(tmp, &tmp->scratch, (size_t)nsm * nsub * (S + 1)))) return rc;
             a.spec = tmp->spec[0];
             a.spec_stride = (long long)nspec * (S + 1);
@@ -515,12 +522,12 @@ int tau_fft_noalloc_impl(int U, int q, int count, const float* blocks, const flo
     a.tw = base;
     a.twlog = kTwLog;
     if (q <= kLogSMax) {
-        const long long per_item = U + 1;
+        const long long per_item = fused_stride(U);
         const int chunk = (int)std::min<long long>(count, avail / per_item);
         for (int i0 = 0; i0 < count; i0 += chunk) {
             const int n = std::min(chunk, count - i0);
             const float* tp = taps + (long long)i0 * ldt;
-            if ((rc = launch_spectra(q, tp, ldt, n, 1, 0, spec, base, st))) return rc;
+            if ((rc = launch_spectra(q, tp, ldt, n, 1, 0, spec, base, st, fused_scale(q), fused_stride(1LL << q)))) return rc;
             a.fin = blocks + (long long)i0 * U;
             a.fout = out + (long long)i0 * U;
             a.ftaps = tp;
@@ -538,7 +545,7 @@ int tau_fft_noalloc_impl(int U, int q, int count, const float* blocks, const flo
         for (int i0 = 0; i0 < count; i0 += chunk) {
             const int n = std::min(chunk, count - i0);
             const float* tp = taps + (long long)i0 * ldt;
-            if ((rc = launch_spectra(kLogSMax, tp, ldt, n, nspec, S, spec, base, st))) return rc;
+            if ((rc = launch_spectra(kLogSMax, tp, ldt, n, nspec, S, spec, base, st, 1.0f, S + 1))) return rc;
             a.fin = blocks + (long long)i0 * U;
             a.fout = out + (long long)i0 * U;
             a.ftaps = tp;
@@ -830,9 +837,9 @@ int create_impl(fi_ctx* c, const float* filters) {
         const long long U = 1LL << q;
         if (q <= kLogSMax) {
             c->spec_split[q] = 1;
-            c->spec_stride[q] = U + 1;
-            if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * (U + 1)))) return rc;
-            if ((rc = launch_spectra(q, c->h, L, (int)(M * D), 1, 0, c->spec[q], c->tw, c->cap))) return rc;
+            c->spec_stride[q] = fused_stride(U);
+            if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * fused_stride(U)))) return rc;
+            if ((rc = launch_spectra(q, c->h, L, (int)(M * D), 1, 0, c->spec[q], c->tw, c->cap, fused_scale(q), fused_stride(1LL << q)))) return rc;
         } else {
             const long long S = 1LL << kLogSMax;
             const int nsub = (int)(U / S);
@@ -840,7 +847,7 @@ int create_impl(fi_ctx* c, const float* filters) {
             c->spec_split[q] = nsub;
             c->spec_stride[q] = (long long)nspec * (S + 1);
             if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * nspec * (S + 1)))) return rc;
-            if ((rc = launch_spectra(kLogSMax, c->h, L, (int)(M * D), nspec, S, c->spec[q], c->tw, c->cap)))
+            if ((rc = launch_spectra(kLogSMax, c->h, L, (int)(M * D), nspec, S, c->spec[q], c->tw, c->cap, 1.0f, S + 1)))
                 return rc;
         }
     }
@@ -1106,6 +1113,8 @@ int fi_tau(int impl, int U, int count, const float* blocks, const float* taps, i
         return set_err(FI_EINVAL, "fi_tau: direct tau limited to U <= %d", 1 << kDirectQMax);
     if (impl == FI_TAU_FFT && (ldt & 1))
         return set_err(FI_EINVAL, "fi_tau: FFT tau reads taps in pairs; ldt must be even");
+    if (impl == FI_TAU_FFT && (((uintptr_t)out & 15) || ((uintptr_t)blocks & 7) || ((uintptr_t)taps & 7)))
+        return set_err(FI_EINVAL, "fi_tau: FFT tau needs out 16-byte and blocks, taps 8-byte aligned");
     if (impl == FI_TAU_FFT && (q < kFftQMin || q > kLogSMax + 2))
         return set_err(FI_EINVAL, "fi_tau: FFT tau needs %d <= U <= %d", 1 << kFftQMin, 1 << (kLogSMax + 2));
     int rc = set_all_attrs();
@@ -1124,6 +1133,8 @@ int fi_tau_fft_noalloc(int U, int count, const float* blocks, const float* taps,
     if (U < 1 || (U & (U - 1)) || count < 1 || !blocks || !taps || !out || ldt < 2 * U || (ldt & 1))
         return set_err(FI_EINVAL, "fi_tau_fft_noalloc: need U a power of two, count >= 1, ldt >= 2U and even, "
                                   "non-NULL pointers");
+    if (((uintptr_t)out & 15) || ((uintptr_t)blocks & 7) || ((uintptr_t)taps & 7))
+        return set_err(FI_EINVAL, "fi_tau_fft_noalloc: needs out 16-byte and blocks, taps 8-byte aligned");
     const int q = ctz64(U);
     if (q < kFftQMin || q > kLogSMax + 2)
         return set_err(FI_EINVAL, "fi_tau_fft_noalloc: U = %d outside [%d, %d], the largest block its fixed "

@@ -25,6 +25,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "fi_fft.cuh"
+
 namespace fi {
 
 // ----------------------------------------------------------------- utilities
@@ -324,17 +326,192 @@ __device__ __forceinline__ void load_half_zero(float2* X, const float* in) {
 }
 
 // ----------------------------------------------------------------- fused FFT tau
-// One gray block per CTA: rFFT_{2U}([block, 0^U]) (.) H_U -> irFFT -> outputs [U, 2U-1]
-// added onto the next U positions.  N = U complex points in shared memory.
-template <int LOGN, int NT>
-__global__ void __launch_bounds__(NT) k_tile_fft(TileArgs a) {
-    extern __shared__ float2 X[];
-    TilePtrs p = tile_ptrs(a, blockIdx.x);
-    load_half_zero<LOGN, NT>(X, p.in);
-    fft_smem<LOGN, NT>(X, a.tw, a.twlog);
-    spectral_multiply<LOGN, NT>(X, p.spec, a.tw, a.twlog);
-    fft_smem<LOGN, NT>(X, a.tw, a.twlog);
-    store_upper_half<LOGN, NT>(X, p.out, a.overwrite);
+// Blocks of one edge U = N for every layer and chain (or stand-alone tau items), one
+// tile per group of T = N / E threads, register-resident radix-16 FFTs (fi_fft.cuh).
+// Forward passes: one radix-R0 pass when log2 N is not a multiple of 4 (twiddle-free,
+// first), then radix-16 passes.  Inverse passes: radix-16 first (the first one
+// continues in registers from the forward's last), the radix-R0 pass last, so that
+// the last pass of each direction is the one that touches global memory only for the
+// half it needs (the zero half of the input is never read, the wrap-around half of
+// the output is never formed).
+template <int LOGN>
+struct FftTile {
+    static constexpr int N = 1 << LOGN;
+    static constexpr int RB = N >= 16 ? 16 : N;           // main radix
+    static constexpr int LOGRB = RB == 16 ? 4 : LOGN;
+    static constexpr int NP = LOGN / LOGRB;                // main-radix passes per FFT
+    static constexpr int LOGR0 = LOGN - NP * LOGRB;
+    static constexpr int R0 = 1 << LOGR0;                  // extra radix (1: none)
+    static constexpr int E = RB;                           // points per thread
+    static constexpr int T = N / E;                        // threads per tile
+    static constexpr int NT = T >= 256 ? T : 256;          // threads per CTA
+    static constexpr int TPC = NT / T;                     // tiles per CTA
+    static constexpr int SME = N + N / 16;                 // padded entries per tile
+    static constexpr bool STAGE_H = N <= 8192;             // spectrum staged in shared memory
+    static constexpr int HST = STAGE_H ? N + 2 : 0;        // staged spectrum entries per tile
+    static constexpr int OST = N / 2;                      // staged old outputs (float2) per tile
+    static constexpr size_t smem = (size_t)TPC * (SME + HST + OST) * sizeof(float2);
+    static constexpr int MINB = NT <= 256 ? 2 : 1;         // CTAs per SM the registers allow
+};
+
+// Asynchronous 16-byte global -> shared copy (cp.async, L2 only), completed by
+// cp_async_wait_all() of the same thread; a barrier then publishes it to the CTA.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// Radix-R Stockham pass whose inputs come from shared memory and whose outputs
+// m >= R/2 (the elements i = b + m N/R >= N/2, i.e. real samples [U, 2U)) are added
+// onto the tile's outputs: y[2(i - N/2)] = Re F[i], y[2(i - N/2) + 1] = -Im F[i].
+template <int LOGN, int R, int BPT, int TWLOG>
+__device__ __forceinline__ void fft_last_pass_store(const float2* X, int t, int T, const float2* __restrict__ tw,
+                                                    float* out, const float2* old_out, int overwrite, bool valid) {
+    constexpr int N = 1 << LOGN, NB = N / R;
+    float2* o2 = reinterpret_cast<float2*>(out);
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) {
+        const int b = t + u * T;
+        float2 v[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) v[r] = X[fft::pad(b + r * NB)];
+        if (NB > 1) fft::apply_twiddles<R, TWLOG>(v, tw, LOGN, b);  // Ns = N/R > b: k = b
+        fft::dft<R>(v);
+        if (valid) {
+#pragma unroll
+            for (int m = R / 2; m < R; ++m) {
+                const float2 F = v[fft::omap<R>(m)];
+                const int q = b + m * NB - N / 2;
+                const float2 y = make_float2(F.x, -F.y);
+                if (overwrite) o2[q] = y;
+                else {
+                    const float2 old = old_out[q];
+                    o2[q] = make_float2(old.x + y.x, old.y + y.y);
+                }
+            }
+        }
+    }
+}
+
+template <int LOGN, int TWLOG>
+__global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_block_fft(TileArgs a) {
+    using G = FftTile<LOGN>;
+    constexpr int N = G::N, RB = G::RB, R0 = G::R0, T = G::T, NP = G::NP, LOGRB = G::LOGRB;
+    extern __shared__ __align__(16) float2 fft_sm[];
+    const int grp = threadIdx.x / T, t = threadIdx.x - grp * T;
+    float2* X = fft_sm + grp * G::SME;
+    float2* Hs = fft_sm + G::TPC * G::SME + grp * G::HST;
+    float2* Os = fft_sm + G::TPC * (G::SME + G::HST) + grp * G::OST;
+    const long long item = (long long)blockIdx.x * G::TPC + grp;
+    const bool valid = item < a.count;
+    const TilePtrs p = tile_ptrs(a, valid ? item : 0);
+    const float2* __restrict__ in2 = reinterpret_cast<const float2*>(p.in);
+    float2 v[1][RB];
+
+    // ---- the spectrum and (when accumulating) the old outputs stream into shared
+    // memory while the forward transform runs
+    if (valid) {
+        if constexpr (G::STAGE_H) {
+            for (int c = t; c < (N + 2) / 2; c += T) cp_async16(Hs + 2 * c, p.spec + 2 * c);
+        }
+        if (!a.overwrite) {
+            for (int c = t; c < N / 4; c += T) cp_async16(Os + 2 * c, p.out + 4 * c);
+        }
+    }
+    cp_async_commit();
+
+    // ---- forward: first pass from global memory (packed block, zero upper half), Ns = 1
+    if constexpr (R0 > 1) {
+        constexpr int BPT = RB / R0, NB = N / R0;
+        float2 w[BPT][R0];
+#pragma unroll
+        for (int u = 0; u < BPT; ++u) {
+            const int b = t + u * T;
+#pragma unroll
+            for (int r = 0; r < R0; ++r) w[u][r] = (r < R0 / 2) ? __ldg(in2 + b + r * NB) : make_float2(0.f, 0.f);
+            fft::dft<R0>(w[u]);
+#pragma unroll
+            for (int m = 0; m < R0; ++m) X[fft::pad(b * R0 + m)] = w[u][fft::omap<R0>(m)];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < NP; ++j) fft::pass<LOGN, RB, 1, TWLOG>(X, v, t, T, G::LOGR0 + j * LOGRB, a.tw);
+    } else {
+        constexpr int NB = N / RB;
+#pragma unroll
+        for (int r = 0; r < RB; ++r) v[0][r] = (r < RB / 2) ? __ldg(in2 + t + r * NB) : make_float2(0.f, 0.f);
+        fft::dft<RB>(v[0]);
+#pragma unroll
+        for (int m = 0; m < RB; ++m) X[fft::pad(t * RB + m)] = v[0][fft::omap<RB>(m)];
+        __syncthreads();
+#pragma unroll
+        for (int j = 1; j < NP; ++j) fft::pass<LOGN, RB, 1, TWLOG>(X, v, t, T, j * LOGRB, a.tw);
+    }
+
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- spectral multiply: this thread holds Z[k], k = t + m N/RB, in v[0][omap(m)];
+    // the partners Z[N-k] are in shared memory (the last pass stored every Z[k]).
+    float2 q[RB];
+    {
+        constexpr int NB = N / RB;
+        const float2* H = G::STAGE_H ? Hs : p.spec;
+        const float2 wb = fft::tw_at<TWLOG>(a.tw, t << (TWLOG - LOGN - 1));  // W_{2N}^t
+#pragma unroll
+        for (int m = 0; m < RB; ++m) {
+            const int k = t + m * NB;
+            const float2 Zk = v[0][fft::omap<RB>(m)];
+            const float2 Zn = X[fft::pad((N - k) & (N - 1))];
+            const float2 Hk = H[k], Hn = H[N - k];
+            const float2 w = fft::cm(wb, fft::w32(m * (16 / RB)));  // W_{2N}^k = (cos, -sin) of pi k / N
+            // Q[k] = conj(Z[k]) (S + sin D) + Z[N-k] (i cos D),  S, D = H[N-k] +- conj H[k]
+            const float2 S = make_float2(Hn.x + Hk.x, Hn.y - Hk.y);
+            const float2 D = make_float2(Hn.x - Hk.x, Hn.y + Hk.y);
+            const float sn = -w.y, cs = w.x;
+            const float2 G1 = make_float2(fmaf(sn, D.x, S.x), fmaf(sn, D.y, S.y));
+            const float2 G2 = make_float2(-cs * D.y, cs * D.x);
+            float2 r = make_float2(fmaf(Zk.x, G1.x, Zk.y * G1.y), fmaf(Zk.x, G1.y, -Zk.y * G1.x));
+            r.x = fmaf(Zn.x, G2.x, fmaf(-Zn.y, G2.y, r.x));
+            r.y = fmaf(Zn.x, G2.y, fmaf(Zn.y, G2.x, r.y));
+            q[m] = r;
+        }
+    }
+    __syncthreads();  // partner reads complete before the inverse overwrites X
+
+    // ---- inverse: first pass in registers (Ns = 1), then shared-memory passes
+    fft::dft<RB>(q);
+    if constexpr (NP == 1 && R0 == 1) {
+        // a single pass: N = RB, the outputs are q[omap(m)] at i = m
+        if (valid) {
+            float2* o2 = reinterpret_cast<float2*>(p.out);
+#pragma unroll
+            for (int m = RB / 2; m < RB; ++m) {
+                const float2 F = q[fft::omap<RB>(m)];
+                const float2 y = make_float2(F.x, -F.y);
+                if (a.overwrite) o2[m - RB / 2] = y;
+                else {
+                    const float2 old = Os[m - RB / 2];
+                    o2[m - RB / 2] = make_float2(old.x + y.x, old.y + y.y);
+                }
+            }
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < RB; ++m) X[fft::pad(t * RB + m)] = q[fft::omap<RB>(m)];
+        __syncthreads();
+        if constexpr (R0 > 1) {
+#pragma unroll
+            for (int j = 1; j < NP; ++j) fft::pass<LOGN, RB, 1, TWLOG>(X, v, t, T, j * LOGRB, a.tw);
+            fft_last_pass_store<LOGN, R0, RB / R0, TWLOG>(X, t, T, a.tw, p.out, Os, a.overwrite, valid);
+        } else {
+#pragma unroll
+            for (int j = 1; j + 1 < NP; ++j) fft::pass<LOGN, RB, 1, TWLOG>(X, v, t, T, j * LOGRB, a.tw);
+            fft_last_pass_store<LOGN, RB, 1, TWLOG>(X, t, T, a.tw, p.out, Os, a.overwrite, valid);
+        }
+    }
 }
 
 // ----------------------------------------------------------------- split FFT tau
@@ -395,13 +572,14 @@ __global__ void __launch_bounds__(NT) k_tile_fft_split(TileArgs a) {
 }
 
 // ----------------------------------------------------------------- filter spectra
-// H[k] = sum_{m<2N} taps[off + m] e^{-2 pi i k m / 2N}, k = 0..N, for every
+// H[k] = scale * sum_{m<2N} taps[off + m] e^{-2 pi i k m / 2N}, k = 0..N, for every
 // (layer, channel) item and every offset e (off = e * offstep).  Run once when a
 // context is created (section "Speicheroptimierung": DFT of the filters per block size).
 template <int LOGN, int NT>
 __global__ void __launch_bounds__(NT) k_spectra(const float* __restrict__ taps, long long ld,
                                                 int nspec, long long offstep, float2* spec,
-                                                const float2* __restrict__ tw, int twlog) {
+                                                const float2* __restrict__ tw, int twlog, float scale,
+                                                long long hstride) {
     extern __shared__ float2 X[];
     constexpr int N = 1 << LOGN;
     const long long item = blockIdx.x / nspec;
@@ -410,14 +588,14 @@ __global__ void __launch_bounds__(NT) k_spectra(const float* __restrict__ taps, 
     for (int m = threadIdx.x; m < N; m += NT) X[m] = t2[m];
     __syncthreads();
     fft_smem<LOGN, NT>(X, tw, twlog);
-    float2* H = spec + ((long long)blockIdx.x) * (N + 1);
+    float2* H = spec + ((long long)blockIdx.x) * hstride;
     for (int k = threadIdx.x; k <= N / 2; k += NT) {
         const int kn = (N - k) & (N - 1);
         float2 Xk, Xn;
         unpack_pair(X[k], X[kn], tw2n<LOGN>(tw, twlog, k), tw2n<LOGN>(tw, twlog, N - k), k == 0,
                     Xk, Xn);
-        H[k] = Xk;
-        H[N - k] = Xn;
+        H[k] = make_float2(Xk.x * scale, Xk.y * scale);
+        H[N - k] = make_float2(Xn.x * scale, Xn.y * scale);
     }
 }
 
