@@ -129,10 +129,11 @@ class FlashInference:
         if not h:
             raise FiError(FI_EINVAL, last_error())
         self._h = h
+        self._lib = lib  # kept for close(), which may run during interpreter shutdown
 
     def close(self):
         if getattr(self, "_h", None):
-            _lib.fi_destroy(self._h)
+            self._lib.fi_destroy(self._h)
             self._h = None
 
     __del__ = close

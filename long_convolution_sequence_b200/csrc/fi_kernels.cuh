@@ -721,25 +721,92 @@ __device__ __forceinline__ int cover_range(int T, int s0, int hi, int* top) {
 
 // One lane of a helper pair: sum over j = lo + part + 2k (k < n2) of in[j] * tp[T - j],
 // where n2 = ceil((hi - lo + 1) / 2) is the same for both lanes, so the two lanes run
-// identical trip counts (no divergence); the odd lane's last term, which would fall
-// one past hi when the range length is odd, is masked.
+// identical trip counts (no divergence).  Full batches of 16 terms per lane, which lie
+// in range for both lanes, issue their 32 shared-memory loads (immediate offsets from
+// two running pointers) before the multiply-adds; one predicated batch takes the
+// remaining 1..16 terms, where a term past hi (the odd lane's last one when the length
+// is odd) loads a valid element and is multiplied by 0.
 __device__ __forceinline__ float dot_pair(const float* in, const float* tp, int T, int lo, int hi, int part) {
     const int n2 = (hi - lo + 2) >> 1;
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    const float* pi = in + lo + part;
+    const float* pt = tp + T - lo - part;
     int k = 0;
-    const int jb = lo + part;
-    for (; k + 4 < n2; k += 4) {  // k .. k+3 < n2 - 1: in range for both lanes
-        const int j = jb + 2 * k;
-        a0 = fmaf(in[j], tp[T - j], a0);
-        a1 = fmaf(in[j + 2], tp[T - j - 2], a1);
-        a2 = fmaf(in[j + 4], tp[T - j - 4], a2);
-        a3 = fmaf(in[j + 6], tp[T - j - 6], a3);
+    for (; k + 16 < n2; k += 16) {
+        float x[16], y[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            x[u] = pi[2 * u];
+            y[u] = pt[-2 * u];
+        }
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+            a0 = fmaf(x[u], y[u], a0);
+            a1 = fmaf(x[u + 1], y[u + 1], a1);
+            a2 = fmaf(x[u + 2], y[u + 2], a2);
+            a3 = fmaf(x[u + 3], y[u + 3], a3);
+        }
+        pi += 32;
+        pt -= 32;
     }
-    for (; k < n2; ++k) {
-        const int j = jb + 2 * k;
-        const bool ok = j <= hi;
-        const int jc = ok ? j : hi;
-        a0 = fmaf(ok ? in[jc] : 0.f, tp[T - jc], a0);
+    if (k < n2) {
+        // terms k .. n2-1 (1..16 of them); the last is past hi for the odd lane of an
+        // odd-length row
+        const int rem = n2 - k;
+        const int last_ok = (lo + part + 2 * (n2 - 1) <= hi) ? rem : rem - 1;
+        float x[16], y[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const bool ok = u < last_ok;
+            const int o = ok ? 2 * u : 0;
+            x[u] = pi[o];
+            y[u] = pt[-o];
+            x[u] = ok ? x[u] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+            a0 = fmaf(x[u], y[u], a0);
+            a1 = fmaf(x[u + 1], y[u + 1], a1);
+            a2 = fmaf(x[u + 2], y[u + 2], a2);
+            a3 = fmaf(x[u + 3], y[u + 3], a3);
+        }
+    }
+    return (a0 + a1) + (a2 + a3);
+}
+
+// The main-loop row of a helper lane's own item with its taps in registers: lane
+// `part` of the pair takes the lags d = 2 + part + 2m, m < nm_me, and adds
+// in[T - d] * tap[d] with tr[m] = tap[2 + part + 2m]; pin = in + T - 2 - part, so term
+// m reads pin[-2m].  nm_both (<= nm_me <= nm_both + 1) terms are valid for both lanes
+// of the pair.  Terms go in blocks of 8 whose loads are issued before their
+// multiply-adds; the block holding the pair's last term is masked per term.  Every
+// index into tr is a compile-time constant, so the taps stay in registers.
+template <int NTR>
+__device__ __forceinline__ float dot_lags(const float* pin, const float (&tr)[NTR], int nm_both, int nm_me) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int b = 0; b < NTR; b += 8) {
+        if (b >= nm_me) break;
+        float x[8];
+        if (b + 8 <= nm_both) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = pin[-2 * (b + u)];
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = b + u < nm_me;
+                const float v = pin[ok ? -2 * (b + u) : 0];
+                x[u] = ok ? v : 0.f;
+            }
+        }
+        a0 = fmaf(x[0], tr[b + 0], a0);
+        a1 = fmaf(x[1], tr[b + 1], a1);
+        a2 = fmaf(x[2], tr[b + 2], a2);
+        a3 = fmaf(x[3], tr[b + 3], a3);
+        a0 = fmaf(x[4], tr[b + 4], a0);
+        a1 = fmaf(x[5], tr[b + 5], a1);
+        a2 = fmaf(x[6], tr[b + 6], a2);
+        a3 = fmaf(x[7], tr[b + 7], a3);
     }
     return (a0 + a1) + (a2 + a3);
 }
@@ -907,6 +974,14 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     geom.tap0 = tap0;
     const PairItem first = decode_item(geom, tid >= 32 ? pair : geom.nitems);
     const bool more = geom.nitems > kWinPairs;  // uniform over the CTA
+    // the helper lane's own item keeps its taps (lags 2 + part + 2m) in registers
+    constexpr int NTR = ((W - 2) / 2 + 7) / 8 * 8;
+    float tr[NTR];
+#pragma unroll
+    for (int m = 0; m < NTR; ++m) {
+        const int d = 2 + part + 2 * m;
+        tr[m] = (tid >= 32 && first.out >= 0 && d < W) ? sm[first.tp + d] : 0.f;
+    }
 
     // ---- tokens
     for (int s = s0; s < s1; ++s) {
@@ -964,7 +1039,18 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             if (T < W) {
                 int top;
                 const int lo = cover_range(T, s0, T, &top);
-                helper_rows(sm, geom, first, more, pair, T, lo, s - 1, kW == 0 && lo == 0, part);
+                // lags 2 .. T - lo of row T (lag 1, the newest input, is the chain's)
+                const int dmax = T - lo;
+                const int nm_me = dmax >= 2 + part ? (dmax - 2 - part) / 2 + 1 : 0;
+                const int nm_both = dmax >= 3 ? (dmax - 3) / 2 + 1 : 0;
+                const bool ow = kW == 0 && lo == 0;
+                float acc = first.out >= 0 ? dot_lags(sm + first.in + T - 2 - part, tr, nm_both, nm_me) : 0.f;
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                if (part == 0 && first.out >= 0) {
+                    float* o = sm + first.out + T;
+                    *o = ow ? acc : *o + acc;
+                }
+                if (more) helper_rows_more(sm, geom, pair, T, lo, s - 1, ow, part);
             }
         }
         __syncthreads();
