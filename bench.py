@@ -38,6 +38,9 @@ WORKLOADS = {
     # the headline stack at a shorter length: a few GB on the device, every launch
     # still larger than L2 (used for profiler captures)
     "short": (18, 1, 864, 1 << 14),
+    # the headline length with fewer channels: every block size up to 2^16 in a few GB
+    # (used for profiler captures of the largest blocks)
+    "narrow": (18, 1, 96, 1 << 17),
 }
 FALLBACK_HBM_GBS = 6650.0
 FP32_LANES_PER_SM = 128
@@ -262,7 +265,7 @@ def main():
     for q in perq:
         impl = info.tau[q]
         name = ("block_direct" if impl == fi.FI_TAU_DIRECT else
-                ("block_split" if q > 14 else "block_fft"))
+                ("block_cluster" if q > int(os.environ.get("FI_FUSED_QMAX", "14")) else "block_fft"))
         classes_q.setdefault(name, set()).add(q)
     ms = max_over_ranks(ms, world, "cuda")
 

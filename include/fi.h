@@ -91,7 +91,7 @@ typedef struct fi_info {
 #define FI_K_TOKEN_STEP 1    /* per-token step kernel: red cells (+ small blocks) */
 #define FI_K_BLOCK_DIRECT 2  /* one block size, every layer and chain, direct tau */
 #define FI_K_BLOCK_FFT 3     /* one block size, every layer and chain, fused FFT tau */
-#define FI_K_BLOCK_SPLIT 4   /* blocks larger than one CTA's FFT, split FFT tau */
+#define FI_K_BLOCK_CLUSTER 4 /* blocks larger than one CTA's FFT: FFT tau on a cluster of CTAs */
 #define FI_K_CLASSES 5
 
 typedef struct fi_trace {
@@ -174,7 +174,7 @@ int fi_debug_schedule(const fi_ctx *ctx, int n, int *U, int *impl, int *src_lo,
 /* Stand-alone tau ([Lem1]) over `count` independent blocks of edge U, all pointers
  * DEVICE memory:  out[i][r] (+)= sum_{j<U} blocks[i][j] * taps[i*ldt + U + r - j],
  * r < U (lags 1 .. 2U-1 of each filter row; ldt >= 2U).  accumulate = 0 overwrites.
- * impl: FI_TAU_DIRECT (U <= 4096) or FI_TAU_FFT (8 <= U <= 65536, ldt even; out
+ * impl: FI_TAU_DIRECT (U <= 4096) or FI_TAU_FFT (8 <= U <= 131072, ldt even; out
  * 16-byte aligned, blocks and taps 8-byte aligned).  Runs on the legacy default stream and
  * returns after completion.  Used to test each tau kernel in isolation. */
 int fi_tau(int impl, int U, int count, const float *blocks, const float *taps, int ldt,
@@ -189,8 +189,8 @@ int fi_tau(int impl, int U, int count, const float *blocks, const float *taps, i
  * Arguments and result are those of fi_tau with impl = FI_TAU_FFT: count blocks of
  * edge U (8 <= U <= 65536, a power of two), taps rows of ldt >= 2U (even) floats,
  * out[i][r] (+)= tau; all pointers DEVICE memory, out 16-byte and blocks, taps
- * 8-byte aligned; the caller owns them.  Every temporary (twiddle table, filter spectra, sub-block spectra) lives
- * in one fixed 8 MiB array in device memory, part of the library image, which every
+ * 8-byte aligned; the caller owns them.  Every temporary (twiddle table, filter
+ * spectra) lives in one fixed 8 MiB array in device memory, part of the library image, which every
  * GPU that loads the library holds until the process exits; large counts are
  * processed in chunks that fit it.  The first call on a device sets that device up
  * (looks up the array's device address and writes the twiddle table with a

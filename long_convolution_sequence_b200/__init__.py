@@ -31,9 +31,9 @@ class fi_info(ctypes.Structure):
                 ("sm_count", ctypes.c_int), ("launches", ctypes.c_longlong)]
 
 
-FI_K_WINDOW, FI_K_TOKEN_STEP, FI_K_BLOCK_DIRECT, FI_K_BLOCK_FFT, FI_K_BLOCK_SPLIT = range(5)
+FI_K_WINDOW, FI_K_TOKEN_STEP, FI_K_BLOCK_DIRECT, FI_K_BLOCK_FFT, FI_K_BLOCK_CLUSTER = range(5)
 FI_K_CLASSES = 5
-KERNEL_CLASS_NAMES = ("window", "token_step", "block_direct", "block_fft", "block_split")
+KERNEL_CLASS_NAMES = ("window", "token_step", "block_direct", "block_fft", "block_cluster")
 
 
 class fi_trace(ctypes.Structure):

@@ -57,8 +57,9 @@ int set_err(int code, const char* fmt, ...) {
     } while (0)
 
 constexpr unsigned kMagic = 0xF1C7A5E5u;
-constexpr int kTwLog = 17;          // twiddle table e^{-2 pi i k / 2^17}
-constexpr int kLogSMax = 14;        // largest FFT held by one CTA: 2^14 complex = 128 KB
+constexpr int kTwLog = 18;          // twiddle table e^{-2 pi i k / 2^18}
+constexpr int kFusedQLimit = 14;    // largest block size whose FFT one CTA can hold (U = 16384)
+constexpr int kFftQMax = 17;        // largest block size served by FFT (clusters of CTAs beyond 2^12)
 constexpr int kFftQMin = 3;         // smallest block size served by FFT (U = 8)
 constexpr int kDirectQMax = 12;     // largest block size served by the direct kernel
 constexpr int kFuseQMax = 4;        // per-token path: blocks up to U = 16 run inside the step kernel
@@ -103,9 +104,6 @@ struct fi_ctx {
     float2* tw = nullptr;            // [2^kTwLog]
     float2* spec[32] = {};           // per block size 2^q
     long long spec_stride[32] = {};  // complex entries per (layer, channel)
-    int spec_split[32] = {};         // nsub for split sizes, 1 for single-CTA sizes, 0 none
-    float2* scratch = nullptr;       // split FFT scratch, split_grid CTAs x 4 x (2^14 + 1)
-    int split_grid = 0;
     int tau[32] = {}, tau_user[32] = {};
     float tau_us[32][2] = {};
     int W = 0, kch = 0, win_ncta = 0;
@@ -247,12 +245,65 @@ int launch_fft_tile(int logn, const TileArgs& a, cudaStream_t st) {
     }
 }
 
-int launch_split_tile(const TileArgs& a, int grid, cudaStream_t st) {
-    constexpr int NT = 1024;
-    const size_t smem = sizeof(float2) << kLogSMax;
-    k_tile_fft_split<kLogSMax, NT><<<grid, NT, smem, st>>>(a);
-    CK(cudaGetLastError());
+// Blocks beyond one CTA: one cluster of NC = 2^LOGNC CTAs per block, 2^LOGN2 points
+// per CTA (U = 2^13 .. 2^17 -> (2, 4096), (4, 4096), (8, 4096), (16, 4096), (16, 8192);
+// clusters of 16 are a non-portable size that B200 supports).
+template <int LOGNC, int LOGN2>
+cudaLaunchConfig_t cluster_config(long long count, cudaStream_t st, cudaLaunchAttribute* at) {
+    using G = ClusterTile<LOGNC, LOGN2>;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(count * G::NC));
+    cfg.blockDim = dim3(G::T);
+    cfg.dynamicSmemBytes = G::smem;
+    cfg.stream = st;
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = G::NC;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+template <int LOGNC, int LOGN2>
+int launch_cluster_t(const TileArgs& a, cudaStream_t st) {
+    cudaLaunchAttribute at[1];
+    cudaLaunchConfig_t cfg = cluster_config<LOGNC, LOGN2>(a.count, st, at);
+    CK(cudaLaunchKernelEx(&cfg, k_block_fft_cluster<LOGNC, LOGN2, kTwLog>, a));
     return FI_OK;
+}
+
+int launch_cluster_tile(int q, const TileArgs& a, cudaStream_t st) {
+    switch (q) {
+        case 13: return launch_cluster_t<1, 12>(a, st);
+        case 14: return launch_cluster_t<2, 12>(a, st);
+        case 15: return launch_cluster_t<3, 12>(a, st);
+        case 16: return launch_cluster_t<4, 12>(a, st);
+        case 17: return launch_cluster_t<4, 13>(a, st);
+        default: return set_err(FI_EINVAL, "no cluster FFT for 2^%d points", q);
+    }
+}
+
+template <int LOGNC, int LOGN2>
+int launch_spectra_cluster_t(const float* taps, long long ld, int count, float2* spec, long long hstride,
+                             const float2* tw, cudaStream_t st, float scale) {
+    cudaLaunchAttribute at[1];
+    cudaLaunchConfig_t cfg = cluster_config<LOGNC, LOGN2>(count, st, at);
+    CK(cudaLaunchKernelEx(&cfg, k_spectra_cluster<LOGNC, LOGN2, kTwLog>, taps, ld, spec, hstride, tw, scale));
+    return FI_OK;
+}
+
+int launch_spectra_cluster(int q, const float* taps, long long ld, int count, float2* spec, long long hstride,
+                           const float2* tw, cudaStream_t st, float scale) {
+    switch (q) {
+        case 13: return launch_spectra_cluster_t<1, 12>(taps, ld, count, spec, hstride, tw, st, scale);
+        case 14: return launch_spectra_cluster_t<2, 12>(taps, ld, count, spec, hstride, tw, st, scale);
+        case 15: return launch_spectra_cluster_t<3, 12>(taps, ld, count, spec, hstride, tw, st, scale);
+        case 16: return launch_spectra_cluster_t<4, 12>(taps, ld, count, spec, hstride, tw, st, scale);
+        case 17: return launch_spectra_cluster_t<4, 13>(taps, ld, count, spec, hstride, tw, st, scale);
+        default: return set_err(FI_EINVAL, "no cluster spectrum kernel for 2^%d points", q);
+    }
 }
 
 int launch_direct_tile(const TileArgs& a, cudaStream_t st) {
@@ -262,11 +313,10 @@ int launch_direct_tile(const TileArgs& a, cudaStream_t st) {
     return FI_OK;
 }
 
-// Spectra for the fused FFT tile kernel carry its 1/(2U) scale (fused_scale); the
-// split kernel's sub-block spectra are unscaled.
+// Spectra of the FFT tau carry the kernels' 1/(2U) scale (fused_scale).  Complex
+// entries per (layer, channel) spectrum: bins 0..U plus one pad entry, so that every
+// spectrum starts on a 16-byte boundary (async copies).
 float fused_scale(int q) { return 1.0f / (2.0f * (float)(1LL << q)); }
-// Complex entries per (layer, channel) spectrum of the fused kernel: bins 0..U plus
-// one pad entry, so that every spectrum starts on a 16-byte boundary (async copies).
 long long fused_stride(long long U) { return U + 2; }
 
 template <int LOGN>
@@ -296,6 +346,33 @@ int launch_spectra(int logn, const float* taps, long long ld, int count, int nsp
         case 14: return launch_spectra_t<14>(taps, ld, count, nspec, offstep, spec, tw, st, scale, hstride);
         default: return set_err(FI_EINVAL, "no spectrum kernel for 2^%d points", logn);
     }
+}
+
+// Largest block size served by the one-CTA FFT tile kernel; larger ones run on a
+// cluster of CTAs.  The choice is fixed per process (FI_FUSED_QMAX overrides it).
+int fused_qmax() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("FI_FUSED_QMAX");
+        const int x = e ? atoi(e) : 14;
+        v = std::max(12, std::min(kFusedQLimit, x));
+    }
+    return v;
+}
+
+// Filter spectra of `count` tap rows (row i at taps + i * ld) for block size 2^q, in
+// the layout the FFT tau of that size reads (natural order for one CTA, CTA order
+// for clusters), stride fused_stride(2^q).
+int make_spectra(int q, const float* taps, long long ld, int count, float2* spec, const float2* tw,
+                 cudaStream_t st) {
+    if (q <= fused_qmax())
+        return launch_spectra(q, taps, ld, count, 1, 0, spec, tw, st, fused_scale(q), fused_stride(1LL << q));
+    return launch_spectra_cluster(q, taps, ld, count, spec, fused_stride(1LL << q), tw, st, fused_scale(q));
+}
+
+// The FFT tau of block size 2^q over a.count tiles.
+int launch_fft(int q, const TileArgs& a, cudaStream_t st) {
+    return q <= fused_qmax() ? launch_fft_tile(q, a, st) : launch_cluster_tile(q, a, st);
 }
 
 template <int W, int MAXM>
@@ -338,6 +415,22 @@ int attr_fft() {
     return FI_OK;
 }
 
+template <int LOGNC, int LOGN2>
+int attr_cluster() {
+    using G = ClusterTile<LOGNC, LOGN2>;
+    CK(cudaFuncSetAttribute(k_block_fft_cluster<LOGNC, LOGN2, kTwLog>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)G::smem));
+    CK(cudaFuncSetAttribute(k_spectra_cluster<LOGNC, LOGN2, kTwLog>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)G::smem));
+    if (G::NC > 8) {
+        CK(cudaFuncSetAttribute(k_block_fft_cluster<LOGNC, LOGN2, kTwLog>,
+                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+        CK(cudaFuncSetAttribute(k_spectra_cluster<LOGNC, LOGN2, kTwLog>,
+                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    }
+    return FI_OK;
+}
+
 template <int W>
 int attr_window() {
     CK(cudaFuncSetAttribute(k_window<W, 8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
@@ -353,10 +446,10 @@ int set_all_attrs() {
     int rc = 0;
     rc |= attr_fft<3>() | attr_fft<4>() | attr_fft<5>() | attr_fft<6>() | attr_fft<7>() | attr_fft<8>();
     rc |= attr_fft<9>() | attr_fft<10>() | attr_fft<11>() | attr_fft<12>() | attr_fft<13>() | attr_fft<14>();
+    rc |= attr_cluster<1, 12>() | attr_cluster<2, 12>() | attr_cluster<3, 12>() | attr_cluster<4, 12>();
+    rc |= attr_cluster<4, 13>();
     rc |= attr_window<32>() | attr_window<64>() | attr_window<128>() | attr_window<256>();
     if (rc) return FI_ECUDA;
-    CK(cudaFuncSetAttribute(k_tile_fft_split<kLogSMax, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            (int)(sizeof(float2) << kLogSMax)));
     CK(cudaFuncSetAttribute(k_tile_direct<kDirectNT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                             (int)(3 * (1 << kDirectQMax) * sizeof(float))));
     done = 1;
@@ -386,17 +479,12 @@ int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st) {
     TileArgs a = stack_tile_args(c, n);
     const int q = ctz64(n);
     const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
-                    : (c->spec_split[q] > 1 ? FI_K_BLOCK_SPLIT : FI_K_BLOCK_FFT);
+                    : (q <= fused_qmax() ? FI_K_BLOCK_FFT : FI_K_BLOCK_CLUSTER);
     LaunchScope scope(c, cls, st, q);
     if (impl == FI_TAU_DIRECT) return launch_direct_tile(a, st);
     a.spec = c->spec[q];
     a.spec_stride = c->spec_stride[q];
-    if (c->spec_split[q] > 1) {
-        a.nsub = c->spec_split[q];
-        a.scratch = c->scratch;
-        return launch_split_tile(a, c->split_grid, st);
-    }
-    return launch_fft_tile(q, a, st);
+    return launch_fft(q, a, st);
 }
 
 int upload_twiddles(fi_ctx* c) {
@@ -432,27 +520,11 @@ int tau_impl(fi_ctx* tmp, int impl, int U, int q, int count, const float* blocks
         if ((rc = upload_twiddles(tmp))) return rc;
         a.tw = tmp->tw;
         a.twlog = kTwLog;
-        if (q <= kLogSMax) {
-            if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * fused_stride(U)))) return rc;
-            if ((rc = launch_spectra(q, taps, ldt, count, 1, 0, tmp->spec[0], tmp->tw, st, fused_scale(q), fused_stride(1LL << q)))) return rc;
-            a.spec = tmp->spec[0];
-            a.spec_stride = fused_stride(U);
-            rc = launch_fft_tile(q, a, st);
-        } else {
-            const long long S = 1LL << kLogSMax;
-            const int nsub = (int)(U / S), nspec = 2 * nsub - 1;
-            int nsm = 0, dev = 0;
-            CK(cudaGetDevice(&dev));
-            CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
-            if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * nspec * (S + 1)))) return rc;
-            if ((rc = launch_spectra(kLogSMax, taps, ldt, count, nspec, S, tmp->spec[0], tmp->tw, st, 1.0f, S + 1))) return rc;
-            if ((rc = dev_alloc(tmp, &tmp->scratch, (size_t)nsm * nsub * (S + 1)))) return rc;
-            a.spec = tmp->spec[0];
-            a.spec_stride = (long long)nspec * (S + 1);
-            a.nsub = nsub;
-            a.scratch = tmp->scratch;
-            rc = launch_split_tile(a, nsm, st);
-        }
+        if ((rc = dev_alloc(tmp, &tmp->spec[0], (size_t)count * fused_stride(U)))) return rc;
+        if ((rc = make_spectra(q, taps, ldt, count, tmp->spec[0], tmp->tw, st))) return rc;
+        a.spec = tmp->spec[0];
+        a.spec_stride = fused_stride(U);
+        rc = launch_fft(q, a, st);
     }
     if (rc) return rc;
     CK(cudaStreamSynchronize(st));
@@ -463,9 +535,9 @@ int tau_impl(fi_ctx* tmp, int impl, int U, int q, int count, const float* blocks
 // Scratch of fi_tau_fft_noalloc: one fixed array per device, part of the library's
 // device image, so it exists from module load to process exit and needs no
 // cudaMalloc.  Layout (complex64 entries): [0, 2^kTwLog) twiddles, written once per
-// device at set-up; then the filter spectra of one chunk of items; then, for block
-// sizes above one CTA's FFT, the split kernel's per-CTA sub-block spectra.
+// device at set-up; then the filter spectra of one chunk of items.
 constexpr int kNoAllocMaxDevices = 64;
+constexpr int kNoAllocQMax = 16;  // largest block (U = 65536) the fixed array serves
 std::mutex g_noalloc_mu;
 float2* g_noalloc_base[kNoAllocMaxDevices] = {};
 
@@ -503,9 +575,8 @@ int noalloc_setup(int dev, float2** base) {
 // items processed in chunks small enough to fit it.
 int tau_fft_noalloc_impl(int U, int q, int count, const float* blocks, const float* taps, int ldt, float* out,
                          int accumulate) {
-    int dev = 0, nsm = 0;
+    int dev = 0;
     CK(cudaGetDevice(&dev));
-    CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
     float2* base = nullptr;
     int rc = noalloc_setup(dev, &base);
     if (rc) return rc;
@@ -521,41 +592,19 @@ int tau_fft_noalloc_impl(int U, int q, int count, const float* blocks, const flo
     a.overwrite = accumulate ? 0 : 1;
     a.tw = base;
     a.twlog = kTwLog;
-    if (q <= kLogSMax) {
-        const long long per_item = fused_stride(U);
-        const int chunk = (int)std::min<long long>(count, avail / per_item);
-        for (int i0 = 0; i0 < count; i0 += chunk) {
-            const int n = std::min(chunk, count - i0);
-            const float* tp = taps + (long long)i0 * ldt;
-            if ((rc = launch_spectra(q, tp, ldt, n, 1, 0, spec, base, st, fused_scale(q), fused_stride(1LL << q)))) return rc;
-            a.fin = blocks + (long long)i0 * U;
-            a.fout = out + (long long)i0 * U;
-            a.ftaps = tp;
-            a.count = n;
-            a.spec = spec;
-            a.spec_stride = per_item;
-            if ((rc = launch_fft_tile(q, a, st))) return rc;
-        }
-    } else {
-        const long long S = 1LL << kLogSMax;
-        const int nsub = (int)(U / S), nspec = 2 * nsub - 1;
-        const long long per_item = (long long)nspec * (S + 1), per_cta = (long long)nsub * (S + 1);
-        const int chunk = (int)std::min<long long>(std::min(count, nsm), avail / (per_item + per_cta));
-        float2* scr = spec + (long long)chunk * per_item;
-        for (int i0 = 0; i0 < count; i0 += chunk) {
-            const int n = std::min(chunk, count - i0);
-            const float* tp = taps + (long long)i0 * ldt;
-            if ((rc = launch_spectra(kLogSMax, tp, ldt, n, nspec, S, spec, base, st, 1.0f, S + 1))) return rc;
-            a.fin = blocks + (long long)i0 * U;
-            a.fout = out + (long long)i0 * U;
-            a.ftaps = tp;
-            a.count = n;
-            a.spec = spec;
-            a.spec_stride = per_item;
-            a.nsub = nsub;
-            a.scratch = scr;
-            if ((rc = launch_split_tile(a, n, st))) return rc;
-        }
+    const long long per_item = fused_stride(U);
+    const int chunk = (int)std::min<long long>(count, avail / per_item);
+    for (int i0 = 0; i0 < count; i0 += chunk) {
+        const int n = std::min(chunk, count - i0);
+        const float* tp = taps + (long long)i0 * ldt;
+        if ((rc = make_spectra(q, tp, ldt, n, spec, base, st))) return rc;
+        a.fin = blocks + (long long)i0 * U;
+        a.fout = out + (long long)i0 * U;
+        a.ftaps = tp;
+        a.count = n;
+        a.spec = spec;
+        a.spec_stride = per_item;
+        if ((rc = launch_fft(q, a, st))) return rc;
     }
     CK(cudaStreamSynchronize(st));
     return FI_OK;
@@ -810,7 +859,6 @@ void free_ctx(fi_ctx* c) {
     cudaFree(c->h);
     cudaFree(c->tw);
     for (int q = 0; q < 32; ++q) cudaFree(c->spec[q]);
-    cudaFree(c->scratch);
     cudaFree(c->sx);
     cudaFree(c->sy);
     for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
@@ -833,29 +881,11 @@ int create_impl(fi_ctx* c, const float* filters) {
     // twiddles from fp64 host trigonometry
     if ((rc = upload_twiddles(c))) return rc;
     // filter spectra for every FFT-served block size
-    for (int q = kFftQMin; q < c->P; ++q) {
+    for (int q = kFftQMin; q < c->P && q <= kFftQMax; ++q) {
         const long long U = 1LL << q;
-        if (q <= kLogSMax) {
-            c->spec_split[q] = 1;
-            c->spec_stride[q] = fused_stride(U);
-            if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * fused_stride(U)))) return rc;
-            if ((rc = launch_spectra(q, c->h, L, (int)(M * D), 1, 0, c->spec[q], c->tw, c->cap, fused_scale(q), fused_stride(1LL << q)))) return rc;
-        } else {
-            const long long S = 1LL << kLogSMax;
-            const int nsub = (int)(U / S);
-            const int nspec = 2 * nsub - 1;
-            c->spec_split[q] = nsub;
-            c->spec_stride[q] = (long long)nspec * (S + 1);
-            if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * nspec * (S + 1)))) return rc;
-            if ((rc = launch_spectra(kLogSMax, c->h, L, (int)(M * D), nspec, S, c->spec[q], c->tw, c->cap, 1.0f, S + 1)))
-                return rc;
-        }
-    }
-    if (c->P - 1 > kLogSMax) {
-        c->split_grid = c->nsm;
-        const long long S = 1LL << kLogSMax;
-        const int nsub_max = (int)((1LL << (c->P - 1)) / S);
-        if ((rc = dev_alloc(c, &c->scratch, (size_t)c->split_grid * nsub_max * (S + 1)))) return rc;
+        c->spec_stride[q] = fused_stride(U);
+        if ((rc = dev_alloc(c, &c->spec[q], (size_t)(M * D) * fused_stride(U)))) return rc;
+        if ((rc = make_spectra(q, c->h, L, (int)(M * D), c->spec[q], c->tw, c->cap))) return rc;
     }
     CK(cudaStreamSynchronize(c->cap));
     if ((rc = choose_window(c))) return rc;
@@ -882,6 +912,11 @@ fi_ctx* fi_create(int layers, int B, int D, int L, const float* filters) {
         return nullptr;
     }
     const long long G = (long long)B * D;
+    if (L > (1 << (kFftQMax + 1))) {
+        set_err(FI_EINVAL, "fi_create: L = %d above %d, the longest sequence whose blocks the FFT tau serves",
+                L, 1 << (kFftQMax + 1));
+        return nullptr;
+    }
     if ((long long)(layers + 1) * G * L > (1LL << 40)) {
         set_err(FI_EINVAL, "fi_create: buffers too large");
         return nullptr;
@@ -1115,15 +1150,14 @@ int fi_tau(int impl, int U, int count, const float* blocks, const float* taps, i
         return set_err(FI_EINVAL, "fi_tau: FFT tau reads taps in pairs; ldt must be even");
     if (impl == FI_TAU_FFT && (((uintptr_t)out & 15) || ((uintptr_t)blocks & 7) || ((uintptr_t)taps & 7)))
         return set_err(FI_EINVAL, "fi_tau: FFT tau needs out 16-byte and blocks, taps 8-byte aligned");
-    if (impl == FI_TAU_FFT && (q < kFftQMin || q > kLogSMax + 2))
-        return set_err(FI_EINVAL, "fi_tau: FFT tau needs %d <= U <= %d", 1 << kFftQMin, 1 << (kLogSMax + 2));
+    if (impl == FI_TAU_FFT && (q < kFftQMin || q > kFftQMax))
+        return set_err(FI_EINVAL, "fi_tau: FFT tau needs %d <= U <= %d", 1 << kFftQMin, 1 << kFftQMax);
     int rc = set_all_attrs();
     if (rc) return rc;
     fi_ctx tmp;  // holds this call's temporary allocations
     rc = tau_impl(&tmp, impl, U, q, count, blocks, taps, ldt, out, accumulate);
     cudaFree(tmp.tw);
     cudaFree(tmp.spec[0]);
-    cudaFree(tmp.scratch);
     tmp.magic = 0;
     return rc;
 }
@@ -1136,9 +1170,9 @@ int fi_tau_fft_noalloc(int U, int count, const float* blocks, const float* taps,
     if (((uintptr_t)out & 15) || ((uintptr_t)blocks & 7) || ((uintptr_t)taps & 7))
         return set_err(FI_EINVAL, "fi_tau_fft_noalloc: needs out 16-byte and blocks, taps 8-byte aligned");
     const int q = ctz64(U);
-    if (q < kFftQMin || q > kLogSMax + 2)
+    if (q < kFftQMin || q > kNoAllocQMax)
         return set_err(FI_EINVAL, "fi_tau_fft_noalloc: U = %d outside [%d, %d], the largest block its fixed "
-                                  "%zu-byte scratch serves", U, 1 << kFftQMin, 1 << (kLogSMax + 2),
+                                  "%zu-byte scratch serves", U, 1 << kFftQMin, 1 << kNoAllocQMax,
                        kNoAllocScratchBytes);
     int rc = set_all_attrs();
     if (rc) return rc;

@@ -103,8 +103,6 @@ struct TileArgs {
     long long spec_stride;  // complex entries per item
     const float2* tw;    // e^{-2 pi i k / 2^twlog}, k < 2^twlog
     int twlog;
-    float2* scratch;     // split FFT: per-CTA spectra of the input sub-blocks
-    int nsub;            // split FFT: U / S
 };
 
 struct TilePtrs {
@@ -510,63 +508,6 @@ __global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_bloc
 #pragma unroll
             for (int j = 1; j + 1 < NP; ++j) fft::pass<LOGN, RB, 1, TWLOG>(X, v, t, T, j * LOGRB, a.tw);
             fft_last_pass_store<LOGN, RB, 1, TWLOG>(X, t, T, a.tw, p.out, Os, a.overwrite, valid);
-        }
-    }
-}
-
-// ----------------------------------------------------------------- split FFT tau
-// Blocks too large for one CTA's shared memory (U = nsub * S, S = 2^LOGS): the U x U
-// block is cut into nsub x nsub sub-blocks of edge S.  Sub-block (i -> o) is the
-// same tau with its lags shifted by (o - i) S, i.e. a 2S circular convolution
-// against the spectrum of taps [e S, e S + 2S) with e = o - i + nsub - 1.  The
-// spectra of the nsub input sub-blocks are kept in a per-CTA scratch area (global
-// memory, read back by the same CTA), the products are summed in the frequency
-// domain, and one inverse FFT per output sub-block finishes it.
-template <int LOGS, int NT>
-__global__ void __launch_bounds__(NT) k_tile_fft_split(TileArgs a) {
-    extern __shared__ float2 X[];
-    constexpr int S = 1 << LOGS;
-    const int nsub = a.nsub;
-    float2* scr = a.scratch + (long long)blockIdx.x * nsub * (S + 1);
-    for (long long item = blockIdx.x; item < a.count; item += gridDim.x) {
-        TilePtrs p = tile_ptrs(a, item);
-        // spectra of the input sub-blocks
-        for (int i = 0; i < nsub; ++i) {
-            load_half_zero<LOGS, NT>(X, p.in + (long long)i * S);
-            fft_smem<LOGS, NT>(X, a.tw, a.twlog);
-            float2* Xi = scr + (long long)i * (S + 1);
-            for (int k = threadIdx.x; k <= S / 2; k += NT) {
-                const int kn = (S - k) & (S - 1);
-                float2 Xk, Xn;
-                unpack_pair(X[k], X[kn], tw2n<LOGS>(a.tw, a.twlog, k),
-                            tw2n<LOGS>(a.tw, a.twlog, S - k), k == 0, Xk, Xn);
-                Xi[k] = Xk;
-                Xi[S - k] = Xn;
-            }
-            __syncthreads();
-        }
-        // output sub-blocks
-        for (int o = 0; o < nsub; ++o) {
-            for (int k = threadIdx.x; k <= S / 2; k += NT) {
-                const int kn = (S - k) & (S - 1);
-                float2 Yk = make_float2(0.f, 0.f), Yn = make_float2(0.f, 0.f);
-                for (int i = 0; i < nsub; ++i) {
-                    const float2* Xi = scr + (long long)i * (S + 1);
-                    const float2* H = p.spec + (long long)(o - i + nsub - 1) * (S + 1);
-                    float2 hk = __ldg(&H[k]), hn = __ldg(&H[S - k]);
-                    float2 xk = Xi[k], xn = Xi[S - k];
-                    Yk = cadd(Yk, cmul(xk, hk));
-                    Yn = cadd(Yn, cmul(xn, hn));
-                }
-                float2 Wk = tw2n<LOGS>(a.tw, a.twlog, k);
-                float2 Wnk = tw2n<LOGS>(a.tw, a.twlog, S - k);
-                X[k] = conjf2(repack(Yk, Yn, Wk));
-                if (k != 0 && kn != k) X[kn] = conjf2(repack(Yn, Yk, Wnk));
-            }
-            __syncthreads();
-            fft_smem<LOGS, NT>(X, a.tw, a.twlog);
-            store_upper_half<LOGS, NT>(X, p.out + (long long)o * S, a.overwrite);
-            __syncthreads();
         }
     }
 }
@@ -1118,3 +1059,6 @@ __global__ void k_read_layer(const float* __restrict__ act, long long L, long lo
 }
 
 }  // namespace fi
+
+// cluster FFT tau (blocks beyond one CTA's shared memory)
+#include "fi_cluster.cuh"

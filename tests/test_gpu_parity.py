@@ -64,7 +64,7 @@ def test_tau_direct_matches_oracle(U):
     assert rel(base.cpu().numpy() - 1.0, ref) < TOL_TF
 
 
-@pytest.mark.parametrize("U", [1 << q for q in range(3, 17)])
+@pytest.mark.parametrize("U", [1 << q for q in range(3, 18)])
 def test_tau_fft_matches_oracle(U):
     rng = np.random.default_rng(U + 1)
     cnt = 3

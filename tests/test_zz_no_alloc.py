@@ -40,9 +40,9 @@ def test_noalloc_rejects_blocks_beyond_its_scratch():
     assert lib.fi_tau_fft_noalloc(8, 0, p, p, 16, p, 0) == fi.FI_EINVAL     # nothing to do
 
 
-# (U, count): counts above what one chunk of the fixed array holds at the split
-# sizes (5 blocks at U = 65536, 11 at U = 32768) so that chunking is exercised
-CASES = [(8, 5), (256, 9), (4096, 4), (16384, 3), (32768, 13), (65536, 7)]
+# (U, count): counts above what one chunk of the fixed array holds at the largest
+# sizes (12 blocks at U = 65536, 24 at U = 32768) so that chunking is exercised
+CASES = [(8, 5), (256, 9), (4096, 4), (16384, 3), (32768, 26), (65536, 13)]
 
 
 @pytest.mark.gpu
