@@ -211,7 +211,7 @@ int dev_alloc(fi_ctx* c, T** p, size_t count) {
 }
 
 size_t win_smem_bytes(int W, int M, int B, int kch) {
-    return (size_t)((M + 1) * kch * B + M * kch) * (W + 2) * sizeof(float);
+    return (size_t)((M + 1) * kch * B + M * kch + M * kch * B) * (W + 4) * sizeof(float);
 }
 
 // chain registers of the window kernel are unrolled up to MAXM layers (18: exact)

@@ -758,6 +758,53 @@ __device__ __forceinline__ float dot_lags(const float* pin, const float (&tr)[NT
     return (a0 + a1) + (a2 + a3);
 }
 
+// Two fp32 multiply-adds in one packed instruction (sm_100): c + a * b per lane.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n.reg .b64 pa, pb, pc;\nmov.b64 pa, {%2, %3};\nmov.b64 pb, {%4, %5};\nmov.b64 pc, {%6, %7};\n"
+        "fma.rn.f32x2 pc, pa, pb, pc;\nmov.b64 {%0, %1}, pc;\n}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
+// The main-loop row of a helper lane's own item, two lags per load and per
+// multiply-add: the lags 2..dmax of row T are taken in pairs (2 + 2k, 3 + 2k); lane
+// `part` takes k = part + 2m, m < nm_me, with trx[m] = (tap[3 + 2k], tap[2 + 2k]) in
+// registers.  The inputs of pair k, positions (T - 3 - 2k, T - 2 - 2k), are one
+// aligned 8-byte load: from the input row when T is odd, else from its copy shifted
+// by one position (pbl points at pair m = 0 of this lane; pair m sits at pbl - 4m).
+// nm_both pairs are whole for both lanes; when dmax is even the last pair's upper
+// lag is past dmax and `last_half` (set on the lane that owns it) drops it.
+template <int NTR2>
+__device__ __forceinline__ float dot_lags2(const float* pbl, const float2 (&trx)[NTR2], int nm_both, int nm_me,
+                                           bool last_half) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int b = 0; b < NTR2; b += 8) {
+        if (b >= nm_me) break;
+        float2 x[8];
+        if (b + 8 <= nm_both) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) x[u] = *reinterpret_cast<const float2*>(pbl - 4 * (b + u));
+        } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = b + u < nm_me;
+                const float2 v = *reinterpret_cast<const float2*>(pbl - (ok ? 4 * (b + u) : 0));
+                x[u] = ok ? v : make_float2(0.f, 0.f);
+                if (last_half && b + u == nm_me - 1) x[u].x = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; u += 2) {
+            a0 = ffma2(x[u], trx[b + u], a0);
+            a1 = ffma2(x[u + 1], trx[b + u + 1], a1);
+        }
+    }
+    return (a0.x + a0.y) + (a1.x + a1.y);
+}
+
 // One helper pair's first (layer, chain) item: shared-memory offsets of its input
 // row, tap row and output row (out < 0: none).  Shapes with more items than pairs
 // hand the pair further items pair + k * kWinPairs, decoded on the fly.
@@ -815,7 +862,9 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     extern __shared__ float4 sm4[];
     float* sm = reinterpret_cast<float*>(sm4);
     constexpr int NT = kWinThreads;
-    constexpr int P = W + 2;  // row pitch: the two lanes of a helper pair and consecutive rows hit distinct banks
+    // row pitch = 4 mod 32: the 8-byte loads of the 16 lanes of half a helper warp
+    // (pair i, lane p at word 132 i - 2p + c) hit 16 distinct bank pairs; 16-byte rows
+    constexpr int P = W + 4;
     const int M = EXACT ? MAXM : a.M;
     const int B = a.B, D = a.D, kch = a.kch;
     const long long L = a.L, G = a.G;
@@ -824,52 +873,41 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     const int ncb = nch * B;
     const int CPB = kch * B;
     const int tap0 = (M + 1) * CPB * P;
+    const int dup0 = tap0 + M * kch * P;  // copies of the input rows (layers 0..M-1), shifted by one
     float* slot = sm;               // [(M+1) * CPB][P]
     float* tap = sm + tap0;         // [M * kch][P]
+    float* dup = sm + dup0;         // [M * CPB][P], dup[x + 1] = activation at window position x
     const long long kW = (a.t0 / W) * (long long)W;  // windows never cross L (W divides L)
     const int s0 = (int)(a.t0 - kW), s1 = (int)(a.t1 - kW);
     const int tid = threadIdx.x;
 
-    // ---- stage the window of every layer and taps 0..W-1 (batched 16-byte loads)
+    // ---- stage the window of every layer and taps 0..W-1: every 16-byte copy in
+    // flight at once (cp.async; rows of W floats at pitch P, 16-byte aligned).
+    // Thread -> (column quad, first row); rows advance by a fixed stride.
     {
-        constexpr int PER = W / 4;
+        constexpr int PER4 = W / 4;
+        constexpr int RSTR = NT / PER4;
         const int rows_slot = (M + 1) * ncb;
-        const int total = (rows_slot + M * nch) * PER;
-        for (int e0 = tid; e0 < total; e0 += NT * 8) {
-            float4 v[8];
-            int dst[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * NT;
-                dst[u] = -1;
-                if (e < total) {
-                    const int row = e / PER, c4 = e - row * PER;
-                    const float* src;
-                    if (row < rows_slot) {
-                        const int l = row / ncb, i = row - l * ncb;
-                        const long long g = (long long)(i / nch) * D + c0 + (i % nch);
-                        src = a.act + ((long long)l * G + g) * L + kW + 4 * c4;
-                        dst[u] = (l * CPB + i) * P + 4 * c4;
-                    } else {
-                        const int r2 = row - rows_slot;
-                        const int l = r2 / nch, ci = r2 - l * nch;
-                        src = a.h + ((long long)l * D + c0 + ci) * L + 4 * c4;
-                        dst[u] = tap0 + (l * kch + ci) * P + 4 * c4;
-                    }
-                    v[u] = __ldg(reinterpret_cast<const float4*>(src));
-                }
+        const int rows = rows_slot + M * nch;
+        const int c4 = tid % PER4;
+        for (int row = tid / PER4; row < rows; row += RSTR) {
+            const float* src;
+            int dst;
+            if (row < rows_slot) {
+                const int l = row / ncb, i = row - l * ncb;
+                const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+                src = a.act + ((long long)l * G + g) * L + kW + 4 * c4;
+                dst = (l * CPB + i) * P + 4 * c4;
+            } else {
+                const int r2 = row - rows_slot;
+                const int l = r2 / nch, ci = r2 - l * nch;
+                src = a.h + ((long long)l * D + c0 + ci) * L + 4 * c4;
+                dst = tap0 + (l * kch + ci) * P + 4 * c4;
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (dst[u] >= 0) {
-                    float* d = sm + dst[u];
-                    d[0] = v[u].x;
-                    d[1] = v[u].y;
-                    d[2] = v[u].z;
-                    d[3] = v[u].w;
-                }
-            }
+            cp_async16(sm + dst, src);
         }
+        cp_async_commit();
+        cp_async_wait_all();
         __syncthreads();
         if (!a.closed) {
             const int steps = s1 - s0;
@@ -884,6 +922,13 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                 const long long g = (long long)(i / nch) * D + c0 + (i % nch);
                 slot[i * P + s0] = a.x[g];
             }
+        }
+        __syncthreads();
+        // shifted copies of the input rows (only positions already final are ever read)
+        for (int e = tid; e < M * ncb * (W - 1); e += NT) {
+            const int row = e / (W - 1), x = e - row * (W - 1);
+            const int l = row / ncb, i = row - l * ncb;
+            dup[(l * CPB + i) * P + x + 1] = slot[(l * CPB + i) * P + x];
         }
         __syncthreads();
     }
@@ -919,13 +964,15 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     geom.tap0 = tap0;
     const PairItem first = decode_item(geom, tid >= 32 ? pair : geom.nitems);
     const bool more = geom.nitems > kWinPairs;  // uniform over the CTA
-    // the helper lane's own item keeps its taps (lags 2 + part + 2m) in registers
-    constexpr int NTR = ((W - 2) / 2 + 7) / 8 * 8;
-    float tr[NTR];
+    // the helper lane's own item keeps its taps in registers, as lag pairs
+    // k = part + 2m: trx[m] = (tap[3 + 2k], tap[2 + 2k])
+    constexpr int NTR2 = ((W - 2) / 4 + 7) / 8 * 8;
+    float2 trx[NTR2];
 #pragma unroll
-    for (int m = 0; m < NTR; ++m) {
-        const int d = 2 + part + 2 * m;
-        tr[m] = (tid >= 32 && first.out >= 0 && d < W) ? sm[first.tp + d] : 0.f;
+    for (int m = 0; m < NTR2; ++m) {
+        const int d = 2 + 2 * (part + 2 * m);
+        const bool ok = tid >= 32 && first.out >= 0;
+        trx[m] = make_float2((ok && d + 1 < W) ? sm[first.tp + d + 1] : 0.f, (ok && d < W) ? sm[first.tp + d] : 0.f);
     }
 
     // ---- tokens
@@ -973,27 +1020,37 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                         av = ahn + e;
                         yl = yh + u;
                         slot[(l * CPB + lane) * P + s] = av;
+                        if (l < M) dup[(l * CPB + lane) * P + s + 1] = av;
                         aprev[l] = av;
                         ah = ahn;
                     }
                 }
                 a.out[(t - a.tx) * G + gch] = yl;
                 if (a.closed) {
-                    if (s + 1 < W) slot[lane * P + s + 1] = av;
-                    else if (t + 1 < L) a.act[gch * L + t + 1] = av;
+                    if (s + 1 < W) {
+                        slot[lane * P + s + 1] = av;
+                        dup[lane * P + s + 2] = av;
+                    } else if (t + 1 < L) {
+                        a.act[gch * L + t + 1] = av;
+                    }
                 }
             }
         } else {
             const int T = s + 1;
             if (T < W) {
                 int top;
-                const int lo = cover_range(T, s0, T, &top);
-                // lags 2 .. T - lo of row T (lag 1, the newest input, is the chain's)
+                // a launch that starts the window holds every block covering T: lo = 0
+                const int lo = s0 == 0 ? 0 : cover_range(T, s0, T, &top);
+                // lags 2 .. T - lo of row T (lag 1, the newest input, is the chain's), in
+                // K = dmax / 2 lag pairs; pair k = part + 2m belongs to this lane
                 const int dmax = T - lo;
-                const int nm_me = dmax >= 2 + part ? (dmax - 2 - part) / 2 + 1 : 0;
-                const int nm_both = dmax >= 3 ? (dmax - 3) / 2 + 1 : 0;
+                const int K = dmax >> 1;
+                const int nm_me = (K - part + 1) >> 1;
+                const int nm_both = ((dmax & 1) ? K : K - 1) >> 1;  // pairs whole for both lanes
+                const bool last_half = ((dmax & 1) == 0) && (((K - 1) & 1) == part);
                 const bool ow = kW == 0 && lo == 0;
-                float acc = first.out >= 0 ? dot_lags(sm + first.in + T - 2 - part, tr, nm_both, nm_me) : 0.f;
+                const float* pb = (T & 1) ? sm + first.in + T - 3 : sm + dup0 + first.in + T - 2;
+                float acc = first.out >= 0 ? dot_lags2(pb - 2 * part, trx, nm_both, nm_me, last_half) : 0.f;
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                 if (part == 0 && first.out >= 0) {
                     float* o = sm + first.out + T;
