@@ -12,7 +12,7 @@ CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 LIB = PKG / "libfi.so"
 SOURCES = [CSRC / "fi_api.cu"]
-DEPS = SOURCES + [CSRC / "fi_kernels.cuh", INCLUDE / "fi.h"]
+DEPS = SOURCES + sorted(CSRC.glob("*.cuh")) + [INCLUDE / "fi.h"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
