@@ -109,6 +109,7 @@ struct fi_ctx {
     int W = 0, kch = 0, win_ncta = 0;
     size_t win_smem = 0;
     int path = FI_PATH_WINDOW, graphs = 1;
+    int pdl = 1;  // window-path launches overlap their start with the predecessor's end
     long long t = 0;
     float* sx = nullptr;  // staging for host inputs
     size_t sx_n = 0;
@@ -218,29 +219,46 @@ size_t win_smem_bytes(int W, int M, int B, int kch) {
 int win_maxm(int M) { return M <= 8 ? 8 : (M == 18 ? 18 : (M <= 20 ? 20 : (M <= 40 ? 40 : 0))); }
 
 // ---------------------------------------------------------------- kernel launchers
+// Launches of the generation path may overlap their start with the predecessor's
+// end (programmatic dependent launch): the kernels read nothing the predecessor
+// writes before griddepcontrol.wait.
+void set_pdl(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* at, int pdl) {
+    if (!pdl) return;
+    at[cfg->numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[cfg->numAttrs].val.programmaticStreamSerializationAllowed = 1;
+    cfg->attrs = at;
+    cfg->numAttrs += 1;
+}
+
 template <int LOGN>
-int launch_fft_tile_t(const TileArgs& a, cudaStream_t st) {
+int launch_fft_tile_t(const TileArgs& a, cudaStream_t st, int pdl) {
     using G = FftTile<LOGN>;
-    const int grid = (a.count + G::TPC - 1) / G::TPC;
-    k_block_fft<LOGN, kTwLog><<<grid, G::NT, G::smem, st>>>(a);
-    CK(cudaGetLastError());
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)((a.count + G::TPC - 1) / G::TPC));
+    cfg.blockDim = dim3(G::NT);
+    cfg.dynamicSmemBytes = G::smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    set_pdl(&cfg, at, pdl);
+    CK(cudaLaunchKernelEx(&cfg, k_block_fft<LOGN, kTwLog>, a));
     return FI_OK;
 }
 
-int launch_fft_tile(int logn, const TileArgs& a, cudaStream_t st) {
+int launch_fft_tile(int logn, const TileArgs& a, cudaStream_t st, int pdl) {
     switch (logn) {
-        case 3: return launch_fft_tile_t<3>(a, st);
-        case 4: return launch_fft_tile_t<4>(a, st);
-        case 5: return launch_fft_tile_t<5>(a, st);
-        case 6: return launch_fft_tile_t<6>(a, st);
-        case 7: return launch_fft_tile_t<7>(a, st);
-        case 8: return launch_fft_tile_t<8>(a, st);
-        case 9: return launch_fft_tile_t<9>(a, st);
-        case 10: return launch_fft_tile_t<10>(a, st);
-        case 11: return launch_fft_tile_t<11>(a, st);
-        case 12: return launch_fft_tile_t<12>(a, st);
-        case 13: return launch_fft_tile_t<13>(a, st);
-        case 14: return launch_fft_tile_t<14>(a, st);
+        case 3: return launch_fft_tile_t<3>(a, st, pdl);
+        case 4: return launch_fft_tile_t<4>(a, st, pdl);
+        case 5: return launch_fft_tile_t<5>(a, st, pdl);
+        case 6: return launch_fft_tile_t<6>(a, st, pdl);
+        case 7: return launch_fft_tile_t<7>(a, st, pdl);
+        case 8: return launch_fft_tile_t<8>(a, st, pdl);
+        case 9: return launch_fft_tile_t<9>(a, st, pdl);
+        case 10: return launch_fft_tile_t<10>(a, st, pdl);
+        case 11: return launch_fft_tile_t<11>(a, st, pdl);
+        case 12: return launch_fft_tile_t<12>(a, st, pdl);
+        case 13: return launch_fft_tile_t<13>(a, st, pdl);
+        case 14: return launch_fft_tile_t<14>(a, st, pdl);
         default: return set_err(FI_EINVAL, "no single-CTA FFT for 2^%d points", logn);
     }
 }
@@ -267,20 +285,21 @@ cudaLaunchConfig_t cluster_config(long long count, cudaStream_t st, cudaLaunchAt
 }
 
 template <int LOGNC, int LOGN2>
-int launch_cluster_t(const TileArgs& a, cudaStream_t st) {
-    cudaLaunchAttribute at[1];
+int launch_cluster_t(const TileArgs& a, cudaStream_t st, int pdl) {
+    cudaLaunchAttribute at[2];
     cudaLaunchConfig_t cfg = cluster_config<LOGNC, LOGN2>(a.count, st, at);
+    set_pdl(&cfg, at, pdl);
     CK(cudaLaunchKernelEx(&cfg, k_block_fft_cluster<LOGNC, LOGN2, kTwLog>, a));
     return FI_OK;
 }
 
-int launch_cluster_tile(int q, const TileArgs& a, cudaStream_t st) {
+int launch_cluster_tile(int q, const TileArgs& a, cudaStream_t st, int pdl) {
     switch (q) {
-        case 13: return launch_cluster_t<1, 12>(a, st);
-        case 14: return launch_cluster_t<2, 12>(a, st);
-        case 15: return launch_cluster_t<3, 12>(a, st);
-        case 16: return launch_cluster_t<4, 12>(a, st);
-        case 17: return launch_cluster_t<4, 13>(a, st);
+        case 13: return launch_cluster_t<1, 12>(a, st, pdl);
+        case 14: return launch_cluster_t<2, 12>(a, st, pdl);
+        case 15: return launch_cluster_t<3, 12>(a, st, pdl);
+        case 16: return launch_cluster_t<4, 12>(a, st, pdl);
+        case 17: return launch_cluster_t<4, 13>(a, st, pdl);
         default: return set_err(FI_EINVAL, "no cluster FFT for 2^%d points", q);
     }
 }
@@ -371,14 +390,21 @@ int make_spectra(int q, const float* taps, long long ld, int count, float2* spec
 }
 
 // The FFT tau of block size 2^q over a.count tiles.
-int launch_fft(int q, const TileArgs& a, cudaStream_t st) {
-    return q <= fused_qmax() ? launch_fft_tile(q, a, st) : launch_cluster_tile(q, a, st);
+int launch_fft(int q, const TileArgs& a, cudaStream_t st, int pdl = 0) {
+    return q <= fused_qmax() ? launch_fft_tile(q, a, st, pdl) : launch_cluster_tile(q, a, st, pdl);
 }
 
 template <int W, int MAXM>
 int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
-    k_window<W, MAXM, MAXM == 18><<<c->win_ncta, kWinThreads, c->win_smem, st>>>(a);
-    CK(cudaGetLastError());
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)c->win_ncta);
+    cfg.blockDim = dim3(kWinThreads);
+    cfg.dynamicSmemBytes = c->win_smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    set_pdl(&cfg, at, c->pdl);
+    CK(cudaLaunchKernelEx(&cfg, k_window<W, MAXM, MAXM == 18>, a));
     return FI_OK;
 }
 
@@ -475,7 +501,7 @@ TileArgs stack_tile_args(const fi_ctx* c, long long n) {
 
 // The gray blocks of every layer released after the n-th token, one launch
 // (section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)").
-int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st) {
+int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st, int pdl = 0) {
     TileArgs a = stack_tile_args(c, n);
     const int q = ctz64(n);
     const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
@@ -484,7 +510,7 @@ int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st) {
     if (impl == FI_TAU_DIRECT) return launch_direct_tile(a, st);
     a.spec = c->spec[q];
     a.spec_stride = c->spec_stride[q];
-    return launch_fft(q, a, st);
+    return launch_fft(q, a, st, pdl);
 }
 
 int upload_twiddles(fi_ctx* c) {
@@ -673,7 +699,7 @@ int enqueue_window_path(fi_ctx* c, long long t0, long long steps, const float* x
         }
         if (rc) return rc;
         if (t1 == (k + 1) * W && t1 < L) {
-            rc = launch_block(c, t1, tau_of(c, ctz64(t1)), st);
+            rc = launch_block(c, t1, tau_of(c, ctz64(t1)), st, c->pdl);
             if (rc) return rc;
         }
         t = t1;
@@ -873,6 +899,7 @@ int create_impl(fi_ctx* c, const float* filters) {
     CK(cudaGetDevice(&c->dev));
     CK(cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev));
     CK(cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking));
+    if (const char* e = getenv("FI_PDL")) c->pdl = atoi(e) ? 1 : 0;
     const long long M = c->M, D = c->D, L = c->L, G = c->G;
     int rc;
     if ((rc = dev_alloc(c, &c->act, (size_t)(M + 1) * G * L))) return rc;

@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
         cp_async_commit();
     }
 
+    grid_dep_wait();  // the block's inputs and old outputs come from the previous launches
     cluster_forward<LOGNC, LOGN2, TWLOG, true>(reinterpret_cast<const float2*>(p.in), X, v, k1, t, a.tw);
     cp_async_wait_all();
     cluster.sync();  // every CTA's Z is in its shared memory, the staged spectrum is complete
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
         }
     }
     cluster.sync();  // partner reads done before X is overwritten; Hs is free
+    grid_dep_launch();
     // this CTA's old outputs (runs [k1 PER, (k1+1) PER) + N2 i, i < NC/2) stream into
     // the spectrum area during the inverse transform
     constexpr int PER = N2 / NC;  // output n2 values of this CTA

@@ -364,6 +364,14 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor in the stream is finishing; it
+// reads nothing the predecessor writes before grid_dep_wait(), which returns once
+// the predecessor has completed and its writes are visible (at once when launched
+// normally).  grid_dep_launch() lets the successor start early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
@@ -416,13 +424,13 @@ __global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_bloc
 
     // ---- the spectrum and (when accumulating) the old outputs stream into shared
     // memory while the forward transform runs
-    if (valid) {
-        if constexpr (G::STAGE_H) {
+    if constexpr (G::STAGE_H) {
+        if (valid)
             for (int c = t; c < (N + 2) / 2; c += T) cp_async16(Hs + 2 * c, p.spec + 2 * c);
-        }
-        if (!a.overwrite) {
-            for (int c = t; c < N / 4; c += T) cp_async16(Os + 2 * c, p.out + 4 * c);
-        }
+    }
+    grid_dep_wait();  // the block's inputs and old outputs come from the previous launches
+    if (valid && !a.overwrite) {
+        for (int c = t; c < N / 4; c += T) cp_async16(Os + 2 * c, p.out + 4 * c);
     }
     cp_async_commit();
 
@@ -484,6 +492,7 @@ __global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_bloc
         }
     }
     __syncthreads();  // partner reads complete before the inverse overwrites X
+    grid_dep_launch();
 
     // ---- inverse: first pass in registers (Ns = 1), then shared-memory passes
     fft::dft<RB>(q);
@@ -883,28 +892,23 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
 
     // ---- stage the window of every layer and taps 0..W-1: every 16-byte copy in
     // flight at once (cp.async; rows of W floats at pitch P, 16-byte aligned).
-    // Thread -> (column quad, first row); rows advance by a fixed stride.
+    // Thread -> (column quad, first row); rows advance by a fixed stride.  The taps
+    // (fixed for the whole generation) go first; the positions, written by the
+    // previous launches, after grid_dep_wait().
     {
         constexpr int PER4 = W / 4;
         constexpr int RSTR = NT / PER4;
         const int rows_slot = (M + 1) * ncb;
-        const int rows = rows_slot + M * nch;
         const int c4 = tid % PER4;
-        for (int row = tid / PER4; row < rows; row += RSTR) {
-            const float* src;
-            int dst;
-            if (row < rows_slot) {
-                const int l = row / ncb, i = row - l * ncb;
-                const long long g = (long long)(i / nch) * D + c0 + (i % nch);
-                src = a.act + ((long long)l * G + g) * L + kW + 4 * c4;
-                dst = (l * CPB + i) * P + 4 * c4;
-            } else {
-                const int r2 = row - rows_slot;
-                const int l = r2 / nch, ci = r2 - l * nch;
-                src = a.h + ((long long)l * D + c0 + ci) * L + 4 * c4;
-                dst = tap0 + (l * kch + ci) * P + 4 * c4;
-            }
-            cp_async16(sm + dst, src);
+        for (int r2 = tid / PER4; r2 < M * nch; r2 += RSTR) {
+            const int l = r2 / nch, ci = r2 - l * nch;
+            cp_async16(sm + tap0 + (l * kch + ci) * P + 4 * c4, a.h + ((long long)l * D + c0 + ci) * L + 4 * c4);
+        }
+        grid_dep_wait();
+        for (int row = tid / PER4; row < rows_slot; row += RSTR) {
+            const int l = row / ncb, i = row - l * ncb;
+            const long long g = (long long)(i / nch) * D + c0 + (i % nch);
+            cp_async16(sm + (l * CPB + i) * P + 4 * c4, a.act + ((long long)l * G + g) * L + kW + 4 * c4);
         }
         cp_async_commit();
         cp_async_wait_all();
@@ -1080,6 +1084,8 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
         }
         __syncthreads();
     }
+
+    grid_dep_launch();
 
     // ---- write the window back (16-byte stores from position s0 rounded down to 4);
     // thread -> (column group, first row), rows advance by a fixed stride
