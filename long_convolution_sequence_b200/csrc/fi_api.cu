@@ -212,7 +212,8 @@ int dev_alloc(fi_ctx* c, T** p, size_t count) {
 }
 
 size_t win_smem_bytes(int W, int M, int B, int kch) {
-    return (size_t)((M + 1) * kch * B + M * kch + M * kch * B) * (W + 4) * sizeof(float);
+    // slot, tap and shifted-copy rows plus the leading zero row, each W + kWinPad floats
+    return (size_t)((M + 1) * kch * B + M * kch + M * kch * B + 1) * (W + kWinPad) * sizeof(float);
 }
 
 // chain registers of the window kernel are unrolled up to MAXM layers (18: exact)
@@ -394,6 +395,13 @@ int launch_fft(int q, const TileArgs& a, cudaStream_t st, int pdl = 0) {
     return q <= fused_qmax() ? launch_fft_tile(q, a, st, pdl) : launch_cluster_tile(q, a, st, pdl);
 }
 
+// chains per CTA fixed at compile time for the 18-layer stack at B = 1 with 6 channels
+// per CTA (864 or fewer channels over 148 SMs), W = 128
+constexpr int kWinCPBT = 6;
+bool win_fixed_geom(const fi_ctx* c, int W) {
+    return W == 128 && c->M == 18 && c->B == 1 && c->kch == kWinCPBT;
+}
+
 template <int W, int MAXM>
 int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
     cudaLaunchConfig_t cfg;
@@ -404,7 +412,13 @@ int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     set_pdl(&cfg, at, c->pdl);
-    CK(cudaLaunchKernelEx(&cfg, k_window<W, MAXM, MAXM == 18>, a));
+    if constexpr (W == 128 && MAXM == 18) {
+        if (win_fixed_geom(c, W)) {
+            CK(cudaLaunchKernelEx(&cfg, k_window<W, MAXM, true, kWinCPBT>, a));
+            return FI_OK;
+        }
+    }
+    CK(cudaLaunchKernelEx(&cfg, k_window<W, MAXM, MAXM == 18, 0>, a));
     return FI_OK;
 }
 
@@ -459,10 +473,13 @@ int attr_cluster() {
 
 template <int W>
 int attr_window() {
-    CK(cudaFuncSetAttribute(k_window<W, 8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<W, 18, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<W, 20, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
-    CK(cudaFuncSetAttribute(k_window<W, 40, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 8, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 18, true, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 20, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    CK(cudaFuncSetAttribute(k_window<W, 40, false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax));
+    if constexpr (W == 128)
+        CK(cudaFuncSetAttribute(k_window<W, 18, true, kWinCPBT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemMax));
     return FI_OK;
 }
 

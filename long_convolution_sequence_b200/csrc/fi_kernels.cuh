@@ -657,6 +657,12 @@ struct WinArgs {
 
 constexpr int kWinThreads = 256;          // warp 0: chain lanes; warps 1..7: helpers
 constexpr int kWinPairs = (kWinThreads - 32) / 2;
+// Every shared-memory row of the window kernel (positions, taps, shifted copies) is
+// followed by kWinPad zero floats, and a zero row precedes the first: a row whose
+// blocks start at window position 0 may then read up to 31 positions below 0 and
+// get zeros, so its lag pairs need no per-term masking.  W + kWinPad = 4 mod 32
+// keeps the helpers' 8-byte loads free of bank conflicts.
+constexpr int kWinPad = 36;
 
 // Lowest input of the blocks released at n in (s0, hi] that cover window position T
 // (window-local), walking n = T, T - lowbit(T), ...; returns -1 if none.  *top gets
@@ -814,6 +820,28 @@ __device__ __forceinline__ float dot_lags2(const float* pbl, const float2 (&trx)
     return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
+// dot_lags2 for a row whose inputs start at window position 0: every lane runs nblk
+// whole blocks of 8 lag pairs; the pairs past the row's last lag (and the upper lag
+// of a partial last pair) read the zero padding below position 0, or meet zero taps
+// past the window, and add exact zeros.
+template <int NTR2>
+__device__ __forceinline__ float dot_lags2_padded(const float* pbl, const float2 (&trx)[NTR2], int nblk) {
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int b = 0; b < NTR2; b += 8) {
+        if (b >= 8 * nblk) break;
+        float2 x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = *reinterpret_cast<const float2*>(pbl - 4 * (b + u));
+#pragma unroll
+        for (int u = 0; u < 8; u += 2) {
+            a0 = ffma2(x[u], trx[b + u], a0);
+            a1 = ffma2(x[u + 1], trx[b + u + 1], a1);
+        }
+    }
+    return (a0.x + a0.y) + (a1.x + a1.y);
+}
+
 // One helper pair's first (layer, chain) item: shared-memory offsets of its input
 // row, tap row and output row (out < 0: none).  Shapes with more items than pairs
 // hand the pair further items pair + k * kWinPairs, decoded on the fly.
@@ -866,16 +894,18 @@ __device__ __forceinline__ void helper_rows(float* sm, const ItemGeom& g, const 
     if (more) helper_rows_more(sm, g, pair, T, lo, hi, ow, part);
 }
 
-template <int W, int MAXM, bool EXACT>
+// CPBT != 0: the launch has B = 1 and kch = CPBT chains per CTA, known at compile
+// time, so every shared-memory row the chain lanes touch sits at an immediate offset.
+template <int W, int MAXM, bool EXACT, int CPBT>
 __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     extern __shared__ float4 sm4[];
-    float* sm = reinterpret_cast<float*>(sm4);
     constexpr int NT = kWinThreads;
     // row pitch = 4 mod 32: the 8-byte loads of the 16 lanes of half a helper warp
-    // (pair i, lane p at word 132 i - 2p + c) hit 16 distinct bank pairs; 16-byte rows
-    constexpr int P = W + 4;
+    // (pair i, lane p at word P i - 2p + c) hit 16 distinct bank pairs; 16-byte rows
+    constexpr int P = W + kWinPad;
+    float* sm = reinterpret_cast<float*>(sm4) + P;  // after the leading zero row
     const int M = EXACT ? MAXM : a.M;
-    const int B = a.B, D = a.D, kch = a.kch;
+    const int B = CPBT ? 1 : a.B, D = a.D, kch = CPBT ? CPBT : a.kch;
     const long long L = a.L, G = a.G;
     const int c0 = blockIdx.x * kch;
     const int nch = min(kch, D - c0);
@@ -910,6 +940,13 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             const long long g = (long long)(i / nch) * D + c0 + (i % nch);
             cp_async16(sm + (l * CPB + i) * P + 4 * c4, a.act + ((long long)l * G + g) * L + kW + 4 * c4);
         }
+        // the zero row before the first row and the padding after every row
+        for (int e = tid; e < P; e += NT) sm[e - P] = 0.f;
+        const int nrows = dup0 / P + M * CPB;
+        for (int e = tid; e < nrows * kWinPad; e += NT) {
+            const int r = e / kWinPad;
+            sm[r * P + W + (e - r * kWinPad)] = 0.f;
+        }
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
@@ -928,11 +965,12 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             }
         }
         __syncthreads();
-        // shifted copies of the input rows (only positions already final are ever read)
-        for (int e = tid; e < M * ncb * (W - 1); e += NT) {
-            const int row = e / (W - 1), x = e - row * (W - 1);
+        // shifted copies of the input rows (only positions already final are ever
+        // read); entry 0 stands for position -1 and is zero
+        for (int e = tid; e < M * ncb * W; e += NT) {
+            const int row = e / W, x = e - row * W;
             const int l = row / ncb, i = row - l * ncb;
-            dup[(l * CPB + i) * P + x + 1] = slot[(l * CPB + i) * P + x];
+            dup[(l * CPB + i) * P + x] = x == 0 ? 0.f : slot[(l * CPB + i) * P + x - 1];
         }
         __syncthreads();
     }
@@ -1049,12 +1087,20 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                 // K = dmax / 2 lag pairs; pair k = part + 2m belongs to this lane
                 const int dmax = T - lo;
                 const int K = dmax >> 1;
-                const int nm_me = (K - part + 1) >> 1;
-                const int nm_both = ((dmax & 1) ? K : K - 1) >> 1;  // pairs whole for both lanes
-                const bool last_half = ((dmax & 1) == 0) && (((K - 1) & 1) == part);
                 const bool ow = kW == 0 && lo == 0;
                 const float* pb = (T & 1) ? sm + first.in + T - 3 : sm + dup0 + first.in + T - 2;
-                float acc = first.out >= 0 ? dot_lags2(pb - 2 * part, trx, nm_both, nm_me, last_half) : 0.f;
+                float acc = 0.f;
+                if (first.out >= 0) {
+                    if (lo == 0) {
+                        // uniform over the CTA; reads reach down to position -31
+                        acc = dot_lags2_padded(pb - 2 * part, trx, (((K + 1) >> 1) + 7) >> 3);
+                    } else {
+                        const int nm_me = (K - part + 1) >> 1;
+                        const int nm_both = ((dmax & 1) ? K : K - 1) >> 1;  // pairs whole for both lanes
+                        const bool last_half = ((dmax & 1) == 0) && (((K - 1) & 1) == part);
+                        acc = dot_lags2(pb - 2 * part, trx, nm_both, nm_me, last_half);
+                    }
+                }
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                 if (part == 0 && first.out >= 0) {
                     float* o = sm + first.out + T;
