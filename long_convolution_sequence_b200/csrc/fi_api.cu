@@ -212,8 +212,10 @@ int dev_alloc(fi_ctx* c, T** p, size_t count) {
 }
 
 size_t win_smem_bytes(int W, int M, int B, int kch) {
-    // slot, tap and shifted-copy rows plus the leading zero row, each W + kWinPad floats
-    return (size_t)((M + 1) * kch * B + M * kch + M * kch * B + 1) * (W + kWinPad) * sizeof(float);
+    // slot, tap and shifted-copy rows plus the leading zero row, each W + kWinPad floats,
+    // and the speculative chain values of two tokens (M x 32 float2 each)
+    return (size_t)((M + 1) * kch * B + M * kch + M * kch * B + 1) * (W + kWinPad) * sizeof(float) +
+           (size_t)2 * M * 32 * sizeof(float2);
 }
 
 // chain registers of the window kernel are unrolled up to MAXM layers (18: exact)

@@ -655,8 +655,8 @@ struct WinArgs {
     int kch;            // channels per CTA
 };
 
-constexpr int kWinThreads = 256;          // warp 0: chain lanes; warps 1..7: helpers
-constexpr int kWinPairs = (kWinThreads - 32) / 2;
+constexpr int kWinThreads = 288;          // warp 0: spec lanes; warp 1: exact lanes; warps 2..8: helpers
+constexpr int kWinPairs = (kWinThreads - 64) / 2;
 // Every shared-memory row of the window kernel (positions, taps, shifted copies) is
 // followed by kWinPad zero floats, and a zero row precedes the first: a row whose
 // blocks start at window position 0 may then read up to 31 positions below 0 and
@@ -791,8 +791,8 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
 // by one position (pbl points at pair m = 0 of this lane; pair m sits at pbl - 4m).
 // nm_both pairs are whole for both lanes; when dmax is even the last pair's upper
 // lag is past dmax and `last_half` (set on the lane that owns it) drops it.
-template <int NTR2>
-__device__ __forceinline__ float dot_lags2(const float* pbl, const float2 (&trx)[NTR2], int nm_both, int nm_me,
+template <int NTR2, int N>
+__device__ __forceinline__ float dot_lags2(const float* pbl, const float2 (&trx)[N], int nm_both, int nm_me,
                                            bool last_half) {
     float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -824,8 +824,8 @@ __device__ __forceinline__ float dot_lags2(const float* pbl, const float2 (&trx)
 // whole blocks of 8 lag pairs; the pairs past the row's last lag (and the upper lag
 // of a partial last pair) read the zero padding below position 0, or meet zero taps
 // past the window, and add exact zeros.
-template <int NTR2>
-__device__ __forceinline__ float dot_lags2_padded(const float* pbl, const float2 (&trx)[NTR2], int nblk) {
+template <int NTR2, int N>
+__device__ __forceinline__ float dot_lags2_padded(const float* pbl, const float2 (&trx)[N], int nblk) {
     float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int b = 0; b < NTR2; b += 8) {
@@ -892,6 +892,17 @@ __device__ __forceinline__ void helper_rows(float* sm, const ItemGeom& g, const 
                                             int pair, int T, int lo, int hi, bool ow, int part) {
     add_row(sm, first, T, lo, hi, ow, part);
     if (more) helper_rows_more(sm, g, pair, T, lo, hi, ow, part);
+}
+
+// One register array serves two roles that never share a thread: the helper lanes keep
+// their tap pairs in it, the chain lanes their per-layer values.  Index i is a
+// compile-time constant wherever these are called (unrolled loops).
+template <int N>
+__device__ __forceinline__ float rget(const float2 (&r)[N], int i) { return (i & 1) ? r[i >> 1].y : r[i >> 1].x; }
+template <int N>
+__device__ __forceinline__ void rset(float2 (&r)[N], int i, float v) {
+    if (i & 1) r[i >> 1].y = v;
+    else r[i >> 1].x = v;
 }
 
 // CPBT != 0: the launch has B = 1 and kch = CPBT chains per CTA, known at compile
@@ -975,12 +986,26 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
         __syncthreads();
     }
 
-    // ---- per-launch setup: chain constants in registers, helper item lists
-    const int lane = tid;
-    const bool chain = tid < 32 && lane < ncb;
+    // ---- per-launch setup.  Warp 0 runs the layer chain of each token speculatively
+    // (spec lanes), warp 1 follows one token behind with the exact activations (exact
+    // lanes), warps 2.. are helper pairs.  Lane c < ncb of warps 0 and 1 owns chain c.
+    const int warp = tid >> 5, lane = tid & 31;
+    const bool chain = warp < 2 && lane < ncb;
     long long gch = 0;
     int cich = 0;
-    float h0r[MAXM], h1r[MAXM], aprev[MAXM + 1];
+    float h0r[MAXM], h1r[MAXM];
+    // Shared register array R: helper lanes hold their tap pairs in R[m]; chain lanes
+    // use it as floats (rget / rset): h2 of layer l at [l - 1], the activations
+    // a^0..a^{M-1} the spec chain used for the previous token at [MAXM + l - 1], and the
+    // exact lanes' e_0..e_{M-1} of the previous token (exact - speculative) at
+    // [2 MAXM + l - 1].
+    constexpr int NTR2 = ((W - 2) / 4 + 7) / 8 * 8;
+    constexpr int NR2 = NTR2 > (3 * MAXM + 1) / 2 ? NTR2 : (3 * MAXM + 1) / 2;
+    float2 R[NR2];
+#pragma unroll
+    for (int m = 0; m < NR2; ++m) R[m] = make_float2(0.f, 0.f);
+    float aMsp = 0.f;      // spec: its last layer's activation (the closed loop's next input)
+    float eM = 0.f;        // exact: e_M of the previous token
     if (chain) {
         cich = lane % nch;
         gch = (long long)(lane / nch) * D + c0 + cich;
@@ -990,12 +1015,13 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             const float* tl = tap + ((lc - 1) * kch + cich) * P;
             h0r[l - 1] = tl[0];
             h1r[l - 1] = tl[1];
+            rset(R, l - 1, tl[2]);
         }
-        // activations of token t0-1 (used only from the second step on)
-#pragma unroll
-        for (int l = 0; l <= MAXM; ++l) aprev[l] = 0.f;
     }
-    const int pair = (tid - 32) >> 1, part = tid & 1;
+    // speculative (pre-activation, activation) of every layer, by token parity:
+    // xch[((s & 1) * M + l - 1) * 32 + lane]
+    float2* xch = reinterpret_cast<float2*>(dup + M * CPB * P);
+    const int pair = (tid - 64) >> 1, part = tid & 1;
     ItemGeom geom;
     geom.nitems = M * ncb;
     geom.ncb = ncb;
@@ -1004,101 +1030,153 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     geom.kch = kch;
     geom.P = P;
     geom.tap0 = tap0;
-    const PairItem first = decode_item(geom, tid >= 32 ? pair : geom.nitems);
+    const PairItem first = decode_item(geom, warp >= 2 ? pair : geom.nitems);
     const bool more = geom.nitems > kWinPairs;  // uniform over the CTA
     // the helper lane's own item keeps its taps in registers, as lag pairs
-    // k = part + 2m: trx[m] = (tap[3 + 2k], tap[2 + 2k])
-    constexpr int NTR2 = ((W - 2) / 4 + 7) / 8 * 8;
-    float2 trx[NTR2];
+    // k = part + 2m: R[m] = (tap[4 + 2k], tap[3 + 2k])
+    if (warp >= 2) {
+        const bool ok = first.out >= 0;
 #pragma unroll
-    for (int m = 0; m < NTR2; ++m) {
-        const int d = 2 + 2 * (part + 2 * m);
-        const bool ok = tid >= 32 && first.out >= 0;
-        trx[m] = make_float2((ok && d + 1 < W) ? sm[first.tp + d + 1] : 0.f, (ok && d < W) ? sm[first.tp + d] : 0.f);
+        for (int m = 0; m < NTR2; ++m) {
+            const int d = 3 + 2 * (part + 2 * m);
+            R[m] = make_float2((ok && d + 1 < W) ? sm[first.tp + d + 1] : 0.f, (ok && d < W) ? sm[first.tp + d] : 0.f);
+        }
     }
 
-    // ---- tokens
-    for (int s = s0; s < s1; ++s) {
+    // ---- tokens.  Iteration s runs the speculative chain of token s (warp 0), the exact
+    // activations of token s - 1 (warp 1) and the helper rows of position s + 1 over
+    // inputs up to s - 2 (lags >= 3); iteration s1 only finishes token s1 - 1.
+    //
+    // Spec lanes: y_l = p_l + h2 a^{l-1}_{s-2} + h1 a^{l-1}_{s-1} + h0 a^{l-1}_s with the
+    // running sum p_l (lags >= 3, from the helpers) and the exact a_{s-2} (written by the
+    // exact lanes one iteration earlier); the two newest inputs are the chain's own
+    // speculative activations, so the chain is one FMA and one SFU tanh per link:
+    //   yh_l = p_l + h2 a^{l-1}_{s-2} + h1 ah^{l-1}_{s-1} + h0 ah^{l-1}_s,  ah^l_s = tanh_sfu(yh_l).
+    // Exact lanes, one token later: with e^l = a^l - ah^l, the exact pre-activation is
+    // y_l = yh_l + u, u = h0 e^{l-1}_s + h1 e^{l-1}_{s-1}; with t = tanh(yh_l) in the
+    // exact form and q = 1 - t^2,
+    //   e^l_s = (t - ah^l_s) + q u (1 - t u)   (Taylor, error ~u^3/3),
+    // a^l_s = ah^l_s + e^l_s.  |e| stays near 2^-11, so the dropped term is below 1e-9:
+    // a^l_s is the exact-form tanh of the exact y_l to rounding.  In the closed loop the
+    // speculative input of layer 1 is the chain's own ah^M_{s-1}, with e^0_s = e^M_{s-1}.
+    for (int s = s0; s <= s1; ++s) {
         const long long t = kW + s;
-        if (tid < 32) {
-            if (chain) {
-                // Running sums of every layer first (independent of the chain), then the
-                // layer chain y_l = p_l + h0_l a_{l-1}, a_l = tanh(y_l).  The chain runs
-                // speculatively on the SFU tanh (one instruction per link):
-                //   yh_l = p_l + h0_l ah_{l-1},  ah_l = tanh_sfu(yh_l),
-                // and the exact activations follow off the critical path: with
-                // t = tanh(yh_l) (exact form), s = 1 - t^2 and u = y_l - yh_l = h0_l e_{l-1},
-                //   e_l = a_l - ah_l = (t - ah_l) + s u (1 - t u)   (Taylor, error ~u^3/3),
-                // and a_l = ah_l + e_l, y_l = yh_l + u.  |e| stays below ~2e-3, so the
-                // dropped term is below 1e-9: a_l is the exact-form tanh of the exact y_l
-                // to rounding.
-                float p[MAXM];
-#pragma unroll
-                for (int l = 1; l <= MAXM; ++l) {
-                    const int lc = l <= M ? l : M;
-                    p[l - 1] = slot[(lc * CPB + lane) * P + s];
-                }
-                const float a0 = slot[lane * P + s];
-                const bool newest = s > s0;  // row 0 of block n = t still lacks a^{l-1}_{t-1}
-                const bool zero = t == 0;    // position 0 has no block: its running sum is 0
+        if (warp == 0) {
+            if (chain && s < s1) {
+                const float* rowp = slot + lane * P + s;  // layer 0, position s
+                const bool newest = s > s0;                       // lag 1 not applied yet
+                const bool lag2 = (s & 1) ? s > s0 + 1 : s > s0;  // lag 2 not applied yet
+                const bool zero = t == 0;                         // position 0 has no block
                 float pp[MAXM];
 #pragma unroll
                 for (int l = 1; l <= MAXM; ++l) {
-                    float v = zero ? 0.f : p[l - 1];
-                    if (newest) v = fmaf(h1r[l - 1], aprev[l - 1], v);
+                    const int lc = l <= M ? l : M;
+                    float v = zero ? 0.f : rowp[lc * CPB * P];
+                    if (newest) v = fmaf(h1r[l - 1], rget(R, MAXM + l - 1), v);
+                    if (lag2) v = fmaf(rget(R, l - 1), rowp[(lc - 1) * CPB * P - 2], v);
                     pp[l - 1] = v;
                 }
-                aprev[0] = a0;
-                float ah = a0, e = 0.f, av = 0.f, yl = 0.f;
+                const float a0 = (a.closed && newest) ? aMsp : rowp[0];
+                float2* xo = xch + (s & 1) * M * 32 + lane;
+                float ah = a0;
 #pragma unroll
                 for (int l = 1; l <= MAXM; ++l) {
                     if (EXACT || l <= M) {
+                        rset(R, MAXM + l - 1, ah);
                         const float yh = fmaf(h0r[l - 1], ah, pp[l - 1]);
-                        const float ahn = sfu_tanh(yh);
-                        const float u = h0r[l - 1] * e;
-                        const float te = act_tanh(yh);
-                        const float se = fmaf(-te, te, 1.f);
-                        e = fmaf(se * u, fmaf(-te, u, 1.f), te - ahn);
-                        av = ahn + e;
-                        yl = yh + u;
-                        slot[(l * CPB + lane) * P + s] = av;
-                        if (l < M) dup[(l * CPB + lane) * P + s + 1] = av;
-                        aprev[l] = av;
-                        ah = ahn;
+                        ah = sfu_tanh(yh);
+                        xo[(l - 1) * 32] = make_float2(yh, ah);
                     }
                 }
-                a.out[(t - a.tx) * G + gch] = yl;
-                if (a.closed) {
-                    if (s + 1 < W) {
-                        slot[lane * P + s + 1] = av;
-                        dup[lane * P + s + 2] = av;
-                    } else if (t + 1 < L) {
-                        a.act[gch * L + t + 1] = av;
+                aMsp = ah;
+            }
+        } else if (warp == 1) {
+            if (s > s0) {
+                const int tau = s - 1;
+                float2* xb = xch + (tau & 1) * M * 32;  // this token's (yh, ah), owned by warp 1 now
+                const float yM = chain ? xb[(M - 1) * 32 + lane].x : 0.f;
+                __syncwarp();
+                // phase 1, every lane: the exact-form tanh t of the speculative pre-activations
+                // of (layer l, chain c) = (q / CPB + 1, q % CPB), q = lane + 32 r, written over yh
+                const int nq = M * CPB;
+                for (int q0 = 0; q0 < nq; q0 += 128) {
+                    float yv[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int q = q0 + lane + 32 * r;
+                        const int l1 = q / CPB;
+                        yv[r] = q < nq ? xb[l1 * 32 + q - l1 * CPB].x : 0.f;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int q = q0 + lane + 32 * r;
+                        const int l1 = q / CPB;
+                        if (q < nq) xb[l1 * 32 + q - l1 * CPB].x = act_tanh(yv[r]);
+                    }
+                }
+                __syncwarp();
+                // phase 2, lane c < ncb: the residual recurrence of chain c through the layers
+                if (chain) {
+                    const bool lag1 = tau > s0;  // the chain used its speculative a_{tau-1}
+                    float e = (a.closed && lag1) ? eM : 0.f;
+                    float* rowo = slot + lane * P + tau;
+                    float* rowd = dup + lane * P + tau + 1;
+                    float2 xv[MAXM];  // (t, ah) of every layer, loaded before the first store
+#pragma unroll
+                    for (int l = 1; l <= MAXM; ++l)
+                        if (EXACT || l <= M) xv[l - 1] = xb[(l - 1) * 32 + lane];
+                    float av = 0.f, u = 0.f;
+#pragma unroll
+                    for (int l = 1; l <= MAXM; ++l) {
+                        if (EXACT || l <= M) {
+                            const float te = xv[l - 1].x, ah = xv[l - 1].y;
+                            const float c1 = lag1 ? h1r[l - 1] * rget(R, 2 * MAXM + l - 1) : 0.f;
+                            u = fmaf(h0r[l - 1], e, c1);
+                            const float se = fmaf(-te, te, 1.f);
+                            const float en = fmaf(se * u, fmaf(-te, u, 1.f), te - ah);
+                            rset(R, 2 * MAXM + l - 1, e);
+                            e = en;
+                            av = ah + en;
+                            rowo[l * CPB * P] = av;
+                            if (l < M) rowd[l * CPB * P] = av;
+                        }
+                    }
+                    eM = e;
+                    a.out[(kW + tau - a.tx) * G + gch] = yM + u;
+                    if (a.closed) {
+                        if (tau + 1 < W) {
+                            slot[lane * P + tau + 1] = av;
+                            dup[lane * P + tau + 2] = av;
+                        } else if (kW + tau + 1 < L) {
+                            a.act[gch * L + kW + tau + 1] = av;
+                        }
                     }
                 }
             }
-        } else {
+        } else if (s < s1) {
             const int T = s + 1;
             if (T < W) {
                 int top;
                 // a launch that starts the window holds every block covering T: lo = 0
                 const int lo = s0 == 0 ? 0 : cover_range(T, s0, T, &top);
-                // lags 2 .. T - lo of row T (lag 1, the newest input, is the chain's), in
-                // K = dmax / 2 lag pairs; pair k = part + 2m belongs to this lane
+                // lags 3 .. T - lo of row T (lags 1 and 2 are the chain's), in K lag pairs
+                // (3 + 2k, 4 + 2k); pair k = part + 2m belongs to this lane.  Pair k reads
+                // positions (T - 4 - 2k, T - 3 - 2k), one aligned 8-byte load: from the
+                // input row when T is even, else from its copy shifted by one position.
                 const int dmax = T - lo;
-                const int K = dmax >> 1;
+                const int K = (dmax - 1) >> 1;
                 const bool ow = kW == 0 && lo == 0;
-                const float* pb = (T & 1) ? sm + first.in + T - 3 : sm + dup0 + first.in + T - 2;
+                const float* pb = (T & 1) ? sm + dup0 + first.in + T - 3 : sm + first.in + T - 4;
                 float acc = 0.f;
                 if (first.out >= 0) {
                     if (lo == 0) {
                         // uniform over the CTA; reads reach down to position -31
-                        acc = dot_lags2_padded(pb - 2 * part, trx, (((K + 1) >> 1) + 7) >> 3);
+                        acc = dot_lags2_padded<NTR2>(pb - 2 * part, R, (((K + 1) >> 1) + 7) >> 3);
                     } else {
                         const int nm_me = (K - part + 1) >> 1;
-                        const int nm_both = ((dmax & 1) ? K : K - 1) >> 1;  // pairs whole for both lanes
-                        const bool last_half = ((dmax & 1) == 0) && (((K - 1) & 1) == part);
-                        acc = dot_lags2(pb - 2 * part, trx, nm_both, nm_me, last_half);
+                        const int nm_both = ((dmax & 1) ? K - 1 : K) >> 1;  // pairs whole for both lanes
+                        const bool last_half = (dmax & 1) && (((K - 1) & 1) == part);
+                        acc = dot_lags2<NTR2>(pb - 2 * part, R, nm_both, nm_me, last_half);
                     }
                 }
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
@@ -1106,22 +1184,28 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                     float* o = sm + first.out + T;
                     *o = ow ? acc : *o + acc;
                 }
-                if (more) helper_rows_more(sm, geom, pair, T, lo, s - 1, ow, part);
+                if (more) helper_rows_more(sm, geom, pair, T, lo, s - 2, ow, part);
             }
         }
         __syncthreads();
     }
 
-    // ---- a launch that stops inside the window completes the blocks it released
+    // ---- a launch that stops inside the window completes the blocks it released:
+    // position s1 still lacks its lag-1 and lag-2 terms (lag 2 only when its block was
+    // released after s0), later positions the rows of blocks released in (s0, s1]
     if (s1 < W && s1 > s0) {
-        if (chain) {
+        if (warp == 0 && chain) {
+            const bool lag2 = (s1 & 1) ? s1 > s0 + 1 : true;
             for (int l = 1; l <= M; ++l) {
                 const float* tl = tap + ((l - 1) * kch + cich) * P;
+                const float* in = slot + ((l - 1) * CPB + lane) * P;
                 float* o = slot + (l * CPB + lane) * P + s1;
-                *o = fmaf(tl[1], slot[((l - 1) * CPB + lane) * P + s1 - 1], *o);
+                float v = fmaf(tl[1], in[s1 - 1], *o);
+                if (lag2) v = fmaf(tl[2], in[s1 - 2], v);
+                *o = v;
             }
         }
-        if (tid >= 32) {
+        if (warp >= 2) {
             for (int T = s1 + 1; T < W; ++T) {
                 int top;
                 const int lo = cover_range(T, s0, s1, &top);

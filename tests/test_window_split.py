@@ -1,0 +1,105 @@
+"""Which (input j, output p) contributions each window launch applies.
+
+The window kernel splits the relaxed tiling's in-window blocks (section
+"Kachelung-Strategie (Algorithmus 1)" of the Flash Inference summary) between three
+roles: the chain lanes add lags 1 and 2 of the current position, the helper pairs add
+the rows of every lag >= 3, and a launch that stops inside the window completes the
+blocks it released.  This restates those decisions (the lag-2 parity rule, the helper
+rows' cover ranges, the completion step) exactly as the kernel takes them and checks,
+against brute force over the tiling, that after every launch of every split of a
+window each pair of a block released so far has been applied exactly once and no
+other pair has."""
+import functools
+import itertools
+import random
+
+import pytest
+
+
+def lowbit(n):
+    return n & -n
+
+
+def block_of(j, p):
+    # the released block n (j < n <= p) whose inputs hold j and whose outputs hold p
+    for n in range(j + 1, p + 1):
+        U = lowbit(n)
+        if n - U <= j < n <= p < n + U:
+            return n
+    raise AssertionError((j, p))
+
+
+def cover_range(T, s0, hi):
+    # lowest input (and highest input) of the blocks released in (s0, hi] covering T
+    lo, n, top = -1, T, -1
+    while n > s0 and n > 0:
+        lon = n - lowbit(n)
+        if n <= hi:
+            if top < 0:
+                top = n - 1
+            lo = lon
+        n = lon
+    return lo, top
+
+
+def lag2_pending(s, s0):
+    # the block holding (s - 2, s) is n = s - 1 for odd s, else n = s
+    return s > s0 + 1 if s & 1 else s > s0
+
+
+def launch(W, s0, s1):
+    added = []
+    for s in range(s0, s1):
+        if s > s0:
+            added.append((s - 1, s))
+        if lag2_pending(s, s0):
+            added.append((s - 2, s))
+        T = s + 1
+        if T < W:
+            lo = 0 if s0 == 0 else cover_range(T, s0, T)[0]
+            added += [(j, T) for j in range(lo, T - 2)]  # lags >= 3
+    if s0 < s1 < W:
+        added.append((s1 - 1, s1))
+        if (s1 & 1) == 0 or s1 > s0 + 1:
+            added.append((s1 - 2, s1))
+        for T in range(s1 + 1, W):
+            lo, top = cover_range(T, s0, s1)
+            if lo >= 0:
+                added += [(j, T) for j in range(lo, top + 1)]
+    return added
+
+
+@functools.lru_cache(maxsize=None)
+def blocks(W):
+    return {(j, p): block_of(j, p) for p in range(W) for j in range(p)}
+
+
+def check(W, splits):
+    applied = {}
+    pts = [0] + list(splits) + [W]
+    for s0, s1 in zip(pts[:-1], pts[1:]):
+        for pr in launch(W, s0, s1):
+            assert 0 <= pr[0] < pr[1] < W, pr
+            applied[pr] = applied.get(pr, 0) + 1
+        want = {pr for pr, n in blocks(W).items() if n <= s1}
+        assert all(c == 1 for c in applied.values()), (splits, s0, s1)
+        assert set(applied) == want, (splits, s0, s1)
+
+
+@pytest.mark.parametrize("W", [32, 64])
+def test_whole_window_and_every_single_split(W):
+    check(W, [])
+    for a in range(1, W):
+        check(W, [a])
+
+
+def test_every_two_way_split():
+    W = 32
+    for a, b in itertools.combinations(range(1, W), 2):
+        check(W, [a, b])
+
+
+def test_random_splits_of_the_128_window():
+    rng = random.Random(7)
+    for _ in range(40):
+        check(128, sorted(rng.sample(range(1, 128), rng.randint(1, 10))))
