@@ -655,8 +655,15 @@ struct WinArgs {
     int kch;            // channels per CTA
 };
 
-constexpr int kWinThreads = 288;          // warp 0: spec lanes; warp 1: exact lanes; warps 2..8: helpers
-constexpr int kWinPairs = (kWinThreads - 64) / 2;
+// Warp 0: spec lanes; warp 1: exact lanes; warps 2..8: helper pairs.  (Warp w runs on
+// scheduler w % 4: the spec warp shares its scheduler with helper warps 4 and 8, the
+// exact warp with helper warp 5; layouts giving the spec or exact warp a scheduler of
+// its own measured slower.)
+constexpr int kWinThreads = 288;
+constexpr int kWinExactWarp = 1;
+constexpr int kWinPairs = 7 * 16;
+__device__ __forceinline__ bool win_helper(int warp) { return warp >= 2; }
+__device__ __forceinline__ int win_helper_index(int warp) { return warp - 2; }
 // Every shared-memory row of the window kernel (positions, taps, shifted copies) is
 // followed by kWinPad zero floats, and a zero row precedes the first: a row whose
 // blocks start at window position 0 may then read up to 31 positions below 0 and
@@ -988,9 +995,9 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
 
     // ---- per-launch setup.  Warp 0 runs the layer chain of each token speculatively
     // (spec lanes), warp 1 follows one token behind with the exact activations (exact
-    // lanes), warps 2.. are helper pairs.  Lane c < ncb of warps 0 and 1 owns chain c.
+    // lanes), warps 2..8 are helper pairs.  Lane c < ncb of warps 0 and 1 owns chain c.
     const int warp = tid >> 5, lane = tid & 31;
-    const bool chain = warp < 2 && lane < ncb;
+    const bool chain = (warp == 0 || warp == kWinExactWarp) && lane < ncb;
     long long gch = 0;
     int cich = 0;
     float h0r[MAXM], h1r[MAXM];
@@ -1019,9 +1026,11 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
         }
     }
     // speculative (pre-activation, activation) of every layer, by token parity:
-    // xch[((s & 1) * M + l - 1) * 32 + lane]
+    // xch[((s & 1) * M + l - 1) * CPB + lane] (dense over (layer, chain): the exact
+    // warp's lanes walk it by q = (l - 1) * CPB + c without bank conflicts)
     float2* xch = reinterpret_cast<float2*>(dup + M * CPB * P);
-    const int pair = (tid - 64) >> 1, part = tid & 1;
+    const bool helper = win_helper(warp);
+    const int pair = win_helper_index(warp) * 16 + (lane >> 1), part = tid & 1;
     ItemGeom geom;
     geom.nitems = M * ncb;
     geom.ncb = ncb;
@@ -1030,11 +1039,11 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
     geom.kch = kch;
     geom.P = P;
     geom.tap0 = tap0;
-    const PairItem first = decode_item(geom, warp >= 2 ? pair : geom.nitems);
+    const PairItem first = decode_item(geom, helper ? pair : geom.nitems);
     const bool more = geom.nitems > kWinPairs;  // uniform over the CTA
     // the helper lane's own item keeps its taps in registers, as lag pairs
     // k = part + 2m: R[m] = (tap[4 + 2k], tap[3 + 2k])
-    if (warp >= 2) {
+    if (helper) {
         const bool ok = first.out >= 0;
 #pragma unroll
         for (int m = 0; m < NTR2; ++m) {
@@ -1077,7 +1086,7 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                     pp[l - 1] = v;
                 }
                 const float a0 = (a.closed && newest) ? aMsp : rowp[0];
-                float2* xo = xch + (s & 1) * M * 32 + lane;
+                float2* xo = xch + (s & 1) * M * CPB + lane;
                 float ah = a0;
 #pragma unroll
                 for (int l = 1; l <= MAXM; ++l) {
@@ -1085,33 +1094,32 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                         rset(R, MAXM + l - 1, ah);
                         const float yh = fmaf(h0r[l - 1], ah, pp[l - 1]);
                         ah = sfu_tanh(yh);
-                        xo[(l - 1) * 32] = make_float2(yh, ah);
+                        xo[(l - 1) * CPB] = make_float2(yh, ah);
                     }
                 }
                 aMsp = ah;
             }
-        } else if (warp == 1) {
+        } else if (warp == kWinExactWarp) {
             if (s > s0) {
                 const int tau = s - 1;
-                float2* xb = xch + (tau & 1) * M * 32;  // this token's (yh, ah), owned by warp 1 now
-                const float yM = chain ? xb[(M - 1) * 32 + lane].x : 0.f;
+                float2* xb = xch + (tau & 1) * M * CPB;  // this token's (yh, ah), owned by warp 1 now
+                const float yM = chain ? xb[(M - 1) * CPB + lane].x : 0.f;
                 __syncwarp();
                 // phase 1, every lane: the exact-form tanh t of the speculative pre-activations
-                // of (layer l, chain c) = (q / CPB + 1, q % CPB), q = lane + 32 r, written over yh
+                // of (layer l, chain c) = (q / CPB + 1, q % CPB), entry q = lane + 32 r,
+                // written over yh
                 const int nq = M * CPB;
                 for (int q0 = 0; q0 < nq; q0 += 128) {
                     float yv[4];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         const int q = q0 + lane + 32 * r;
-                        const int l1 = q / CPB;
-                        yv[r] = q < nq ? xb[l1 * 32 + q - l1 * CPB].x : 0.f;
+                        yv[r] = q < nq ? xb[q].x : 0.f;
                     }
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         const int q = q0 + lane + 32 * r;
-                        const int l1 = q / CPB;
-                        if (q < nq) xb[l1 * 32 + q - l1 * CPB].x = act_tanh(yv[r]);
+                        if (q < nq) xb[q].x = act_tanh(yv[r]);
                     }
                 }
                 __syncwarp();
@@ -1124,16 +1132,20 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                     float2 xv[MAXM];  // (t, ah) of every layer, loaded before the first store
 #pragma unroll
                     for (int l = 1; l <= MAXM; ++l)
-                        if (EXACT || l <= M) xv[l - 1] = xb[(l - 1) * 32 + lane];
+                        if (EXACT || l <= M) xv[l - 1] = xb[(l - 1) * CPB + lane];
                     float av = 0.f, u = 0.f;
 #pragma unroll
                     for (int l = 1; l <= MAXM; ++l) {
                         if (EXACT || l <= M) {
+                            // with u = h0 e + c1: q u = (q h0) e + q c1 and 1 - t u =
+                            // (-t h0) e + (1 - t c1), so each link is two dependent FMAs
                             const float te = xv[l - 1].x, ah = xv[l - 1].y;
                             const float c1 = lag1 ? h1r[l - 1] * rget(R, 2 * MAXM + l - 1) : 0.f;
-                            u = fmaf(h0r[l - 1], e, c1);
                             const float se = fmaf(-te, te, 1.f);
-                            const float en = fmaf(se * u, fmaf(-te, u, 1.f), te - ah);
+                            const float w = fmaf(se * h0r[l - 1], e, se * c1);
+                            const float z = fmaf(-te * h0r[l - 1], e, fmaf(-te, c1, 1.f));
+                            if (l == M) u = fmaf(h0r[l - 1], e, c1);
+                            const float en = fmaf(w, z, te - ah);
                             rset(R, 2 * MAXM + l - 1, e);
                             e = en;
                             av = ah + en;
@@ -1153,7 +1165,7 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                     }
                 }
             }
-        } else if (s < s1) {
+        } else if (helper && s < s1) {
             const int T = s + 1;
             if (T < W) {
                 int top;
@@ -1205,7 +1217,7 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
                 *o = v;
             }
         }
-        if (warp >= 2) {
+        if (helper) {
             for (int T = s1 + 1; T < W; ++T) {
                 int top;
                 const int lo = cover_range(T, s0, s1, &top);
