@@ -217,7 +217,14 @@ def main():
                     help="skip the extra traced step that times each kernel class")
     ap.add_argument("--path", choices=("window", "token"), default="window")
     ap.add_argument("--graphs", type=int, default=1)
+    ap.add_argument("--sweep", action="store_true",
+                    help="the configuration sweep (18 layers; B, D, L grids): one JSON line per point")
+    ap.add_argument("--sweep-b", default="1,2,4,8")
+    ap.add_argument("--sweep-d", default="256,512,768,1024")
+    ap.add_argument("--sweep-l", default="12,14,16,18", help="log2 L values")
     args = ap.parse_args()
+    if args.sweep:
+        return bench_sweep(args)
     M, B, D, L = WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -405,6 +412,96 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def sweep_need_bytes(M, B, D, L):
+    """Device memory a sweep point needs: the context's filters plus their spectra
+    (about 3 M D L floats), its halved-layout buffers ((M+1) B D L floats), and the
+    device copy of the filters it is created from (M D L floats)."""
+    return 4 * L * D * (4 * M + (M + 1) * B)
+
+
+def sweep_filters(M, D, L, seed=0):
+    """Filters of the sweep drawn on the device with the same law as the headline's
+    (h[c, k] = N(0,1) exp(-a_c k) / sqrt(32), a_c ~ U(0.001, 0.05), independent per
+    layer), from torch's seeded CUDA generator: the 2^18-tap filters of the largest
+    points would take minutes on the host."""
+    import torch
+    h = torch.empty((M, D, L), device="cuda", dtype=torch.float32)
+    k = torch.arange(L, device="cuda", dtype=torch.float32)
+    for l in range(M):
+        g = torch.Generator(device="cuda")
+        g.manual_seed(1_000_003 * seed + l)
+        a = torch.empty(D, device="cuda").uniform_(0.001, 0.05, generator=g)
+        h[l].normal_(generator=g)
+        h[l] *= torch.exp(-a[:, None] * k[None, :]) / math.sqrt(32.0)
+    return h
+
+
+def bench_sweep(args):
+    """Configuration sweep on the synthetic mixer stack: 18 layers, B, D, L over the
+    given grids.  Per point: one warm-up and one timed closed-loop generation (CUDA
+    events), the tile-size histogram of the schedule, and the tau implementation
+    chosen per block size.  Points whose memory need exceeds the free device memory
+    are reported as not fitting."""
+    import torch
+    import long_convolution_sequence_b200 as fi
+    M = 18
+    hbm, peak_kind, sm_mhz = peaks()
+    names = {fi.FI_TAU_DIRECT: "direct", fi.FI_TAU_FFT: "fft"}
+    for B in [int(v) for v in args.sweep_b.split(",")]:
+        for D in [int(v) for v in args.sweep_d.split(",")]:
+            for P in [int(v) for v in args.sweep_l.split(",")]:
+                L = 1 << P
+                line = {"metric": "sweep point: mixer tokens/s", "layers": M, "B": B, "D": D, "L": L}
+                need = sweep_need_bytes(M, B, D, L)
+                free, _ = torch.cuda.mem_get_info()
+                if need > 0.85 * free:
+                    line.update({"fits": False, "need_gb": round(need / 1e9, 1), "free_gb": round(free / 1e9, 1)})
+                    print(json.dumps(line), flush=True)
+                    continue
+                h = sweep_filters(M, D, L)
+                x0 = torch.from_numpy(synth_start(B, D)).cuda()
+                t0 = time.perf_counter()
+                ctx = fi.FlashInference(M, B, D, L, h)
+                t_create = time.perf_counter() - t0
+                del h
+                torch.cuda.empty_cache()
+                info = ctx.info()
+                out = torch.empty((L, B, D), device="cuda")
+                ctx.reset()
+                ctx.generate(x0, L, out)
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ctx.reset()
+                ev0.record()
+                ctx.generate(x0, L, out)
+                ev1.record()
+                torch.cuda.synchronize()
+                ms = ev0.elapsed_time(ev1)
+                byts, flops = model_bytes_flops(M, B, D, L)
+                fp32_peak = info.sm_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6
+                t_roof = max(byts / (hbm * 1e9), flops / fp32_peak)
+                cls = ["block_cluster" if q > int(os.environ.get("FI_FUSED_QMAX", "14")) and info.tau[q] == fi.FI_TAU_FFT
+                       else names.get(info.tau[q], str(info.tau[q])) for q in range(P)]
+                line.update({
+                    "fits": True, "ms": round(ms, 3), "value": round(B * L / (ms / 1e3), 1),
+                    "roofline_frac": round(t_roof * 1e3 / ms, 4),
+                    "path": "window W=%d" % info.window if info.window else "per-token",
+                    "tile_histogram": {str(1 << q): 1 << (P - 1 - q) for q in range(P)},
+                    "tau": {str(1 << q): cls[q] for q in range(P)},
+                    "create_s": round(t_create, 2), "device_gb": round(info.device_bytes / 1e9, 2),
+                    "finite": bool(torch.isfinite(out).all().item()),
+                })
+                print(json.dumps(line), flush=True)
+                ctx.close()
+                del out
+                torch.cuda.empty_cache()
+    return 0
+
+
+def synth_start(B, D):
+    from long_convolution_sequence_b200 import synth
+    return synth.start_token(B, D, seed=0)
 
 
 def bench_reference(args, M, B, D, L, synth):

@@ -819,22 +819,33 @@ int choose_window(fi_ctx* c) {
     const char* env = getenv("FI_WINDOW");
     int forced = env ? atoi(env) : 0;
     if (c->B > 32) return FI_OK;  // chain lanes: one warp per CTA
-    int kch = (int)((c->D + c->nsm - 1) / c->nsm);
-    if (kch * c->B > 32) kch = std::max(1, 32 / c->B);
-    const int ncta = (c->D + kch - 1) / kch;
-    const int per_sm = (ncta + c->nsm - 1) / c->nsm;
     if (!win_maxm(c->M)) return FI_OK;
+    int kch0 = (int)((c->D + c->nsm - 1) / c->nsm);
+    if (kch0 * c->B > 32) kch0 = std::max(1, 32 / c->B);
+    // The window kernel holds one CTA per SM (its registers) and its CTAs never wait on
+    // one another, so a launch may take several waves.  Per window W, the most channels
+    // per CTA whose rows fit gives the fewest waves; a wave costs about the same per
+    // token at any W, plus a per-launch overhead (~16 tokens' worth) that W amortises.
     const int cand[] = {128, 64, 256, 32};
+    double best = 1e300;
     for (int W : cand) {
         if (forced && W != forced) continue;
         if (W > c->L) continue;
-        size_t sm = win_smem_bytes(W, c->M, c->B, kch);
-        if (sm > kSmemMax || sm * per_sm > 228 * 1024) continue;
-        c->W = W;
-        c->kch = kch;
-        c->win_ncta = ncta;
-        c->win_smem = sm;
-        return FI_OK;
+        for (int kch = kch0; kch >= 1; --kch) {
+            const size_t sm = win_smem_bytes(W, c->M, c->B, kch);
+            if (sm > kSmemMax) continue;
+            const int ncta = (c->D + kch - 1) / kch;
+            const int waves = (ncta + c->nsm - 1) / c->nsm;
+            const double cost = waves * (1.0 + 16.0 / W);
+            if (cost < best - 1e-9) {
+                best = cost;
+                c->W = W;
+                c->kch = kch;
+                c->win_ncta = ncta;
+                c->win_smem = sm;
+            }
+            break;
+        }
     }
     return FI_OK;  // W = 0: window path unavailable, per-token path only
 }

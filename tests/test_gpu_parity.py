@@ -150,6 +150,25 @@ def test_teacher_forced_all_layers(M, B, D, L, W, window):
         assert np.abs(a[l] - np.tanh(ref["y_all"][l - 1])).max() < TOL_TF * rms, l
 
 
+def test_window_launch_of_several_waves(window):
+    # 18 layers, B = 4, D = 512 at W = 64: the rows of 4 channels per CTA do not fit in
+    # shared memory, so the window launch holds 3 channels per CTA: 171 CTAs, more than
+    # the SMs, in two waves
+    M, B, D, L = 18, 4, 512, 512
+    window(64)
+    h = synth.filters(M, D, L, seed=4)
+    x = synth.inputs(L, B, D, seed=4)
+    ref = oracle.stack(h, x, want=("y_last",))
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        info = ctx.info()
+        assert info.window == 64
+        kch = info.chains_per_cta // B
+        assert -(-D // kch) > info.sm_count
+        y = np.empty((L, B, D), np.float32)
+        ctx.forward(x, L, y)
+    assert rel(y, ref["y_last"]) < TOL_TF
+
+
 @pytest.mark.parametrize("M,B,D,L,W", [(1, 1, 16, 1024, None), (3, 2, 6, 4096, 64), (18, 1, 8, 4096, None)])
 def test_closed_loop_matches_oracle(M, B, D, L, W, window):
     window(W)
