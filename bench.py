@@ -222,9 +222,14 @@ def main():
     ap.add_argument("--sweep-b", default="1,2,4,8")
     ap.add_argument("--sweep-d", default="256,512,768,1024")
     ap.add_argument("--sweep-l", default="12,14,16,18", help="log2 L values")
+    ap.add_argument("--baseline", choices=("lazy", "eager"),
+                    help="time the pages' Lazy or Eager baseline on this device next to the tiled path "
+                         "(default workload: short)")
     args = ap.parse_args()
     if args.sweep:
         return bench_sweep(args)
+    if args.baseline:
+        return bench_baseline(args)
     M, B, D, L = WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -496,6 +501,55 @@ def bench_sweep(args):
                 ctx.close()
                 del out
                 torch.cuda.empty_cache()
+    return 0
+
+
+def bench_baseline(args):
+    """The pages' parallel Lazy or Eager baseline (FI_PATH_LAZY / FI_PATH_EAGER) timed
+    on this device beside the tiled window path, same workload, same process: one
+    closed-loop generation each after warm-up, CUDA events.  Both baselines cost O(L^2)
+    per channel-layer, so the headline length (2^17) is out of reach in minutes; the
+    default workload is the headline stack at L = 2^14, and the line also carries the
+    baseline's time scaled to L = 2^17 by the L^2 law (labelled as extrapolated)."""
+    import torch
+    import long_convolution_sequence_b200 as fi
+    from long_convolution_sequence_b200 import synth
+    wl = args.workload if args.workload != "headline" else "short"
+    M, B, D, L = WORKLOADS[wl]
+    h = synth.filters(M, D, L, seed=0)
+    x0 = torch.from_numpy(synth.start_token(B, D, seed=0)).cuda()
+    out = torch.empty((L, B, D), device="cuda")
+    ctx = fi.FlashInference(M, B, D, L, h)
+
+    def timed(n):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for _ in range(n):
+            ctx.reset()
+            ctx.generate(x0, L, out)
+        ev1.record()
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1) / n
+
+    timed(3)
+    fi_ms = timed(3)
+    ctx.reset()
+    ctx.set_path(fi.FI_PATH_LAZY if args.baseline == "lazy" else fi.FI_PATH_EAGER)
+    ctx.generate(x0, min(L, 256), out)  # warm-up of the baseline's kernels
+    torch.cuda.synchronize()
+    base_ms = timed(1)
+    finite = bool(torch.isfinite(out).all().item())
+    ctx.close()
+    scale = (float(1 << 17) / L) ** 2
+    line = {"metric": "mixer tokens/s (B*L/time), %s baseline on this device" % args.baseline,
+            "impl": args.baseline + "_gpu", "value": round(B * L / (base_ms / 1e3), 1),
+            "unit": "tokens/s", "ms_per_generation": round(base_ms, 3),
+            "tiled_value": round(B * L / (fi_ms / 1e3), 1), "tiled_ms_per_generation": round(fi_ms, 3),
+            "tiled_speedup": round(base_ms / fi_ms, 2),
+            "extrapolated_ms_at_L_2^17": round(base_ms * scale, 1) if L < (1 << 17) else None,
+            "finite": finite, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl, "layers": M, "B": B, "D": D, "L": L}}
+    print(json.dumps(line), flush=True)
     return 0
 
 

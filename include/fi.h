@@ -21,6 +21,9 @@
  *   [Circ]  section "Zirkulaere Faltungs-Trick": a 2U circular convolution suffices
  *   [Impl]  section "Implementierungsdetails": CUDA graphs per token, FFT precompute,
  *           Hybrid choice of the tau implementation by block size
+ *   [Base]  section "Kern-Algorithmus: Relaxierte Polynominterpolation", part 1 (the
+ *           Lazy and Eager evaluations) and "Vergleichsmethoden" (their parallel
+ *           versions as the baselines)
  *   [Lem1]  section "Beitrags-Aggregations-Definition", Lemma 1:
  *           tau(y,[l,r],rho,[l',r'])_t = sum_{i=l}^{r} y_i rho_{t-i}
  *
@@ -69,6 +72,10 @@ extern "C" {
                                tokens (red cells + all blocks smaller than W, in shared
                                memory), one launch per larger block */
 #define FI_PATH_TOKEN 1     /* the pages' design: one launch sequence (graph) per token */
+#define FI_PATH_LAZY 2      /* baseline ([Base] "Lazy"): y^l_t summed over the whole history
+                               when token t needs it, O(t) per token; one launch per token */
+#define FI_PATH_EAGER 3     /* baseline ([Base] "Eager"): each activation pushed onto every
+                               later position as soon as it is known, O(L-t) per token */
 
 typedef struct fi_ctx fi_ctx;
 
@@ -143,7 +150,12 @@ int fi_read_layer(fi_ctx *ctx, int layer, int t0, int t1, float *dst);
 /* Use `stream` (a cudaStream_t, NULL = legacy default stream) for all later work. */
 int fi_set_stream(fi_ctx *ctx, void *stream);
 
-/* Choose the execution path (FI_PATH_WINDOW or FI_PATH_TOKEN). */
+/* Choose the execution path (FI_PATH_*).  The two tiled paths (WINDOW, TOKEN) share
+   their buffer state and may be switched at any token; LAZY and EAGER keep their own
+   state, so a change to or from them is accepted only at t = 0 (after fi_create or
+   fi_reset), else FI_EINVAL.  LAZY and EAGER are the pages' parallel baselines: the
+   part of token t that does not depend on its own layer chain runs for every layer at
+   once; they take no graphs and record no trace. */
 int fi_set_path(fi_ctx *ctx, int path);
 
 /* Enable (1) or disable (0) replay of captured CUDA graphs ([Impl]). */

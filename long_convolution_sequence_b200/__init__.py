@@ -14,7 +14,7 @@ _LIB_PATH = Path(__file__).resolve().parent / "libfi.so"
 
 FI_OK, FI_EINVAL, FI_ECAPACITY, FI_ENOMEM, FI_ECUDA, FI_ESTATE = 0, -1, -2, -3, -4, -5
 FI_TAU_AUTO, FI_TAU_DIRECT, FI_TAU_FFT = 0, 1, 2
-FI_PATH_WINDOW, FI_PATH_TOKEN = 0, 1
+FI_PATH_WINDOW, FI_PATH_TOKEN, FI_PATH_LAZY, FI_PATH_EAGER = 0, 1, 2, 3
 
 
 class FiError(RuntimeError):

@@ -745,7 +745,38 @@ void drop_graphs(fi_ctx* c) {
 
 // Run a launch sequence, from a captured graph when enabled (section
 // "Implementierungsdetails": CUDA graphs remove the per-launch CPU overhead).
+// The Lazy / Eager baselines: one launch per token, one CTA per chain.
+int run_baseline(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed) {
+    const bool eager = c->path == FI_PATH_EAGER;
+    if (eager && t0 == 0)  // running sums of layers 1..M start at zero
+        CK(cudaMemsetAsync(c->act + c->G * c->L, 0, sizeof(float) * c->M * c->G * c->L, c->stream));
+    BaseArgs a;
+    a.act = c->act;
+    a.h = c->h;
+    a.M = c->M;
+    a.D = c->D;
+    a.G = c->G;
+    a.L = c->L;
+    a.tx = t0;
+    a.x = x;
+    a.out = out;
+    a.closed = closed;
+    const int threads = eager ? 512 : 32 * std::min(c->M, 32);
+    const size_t smem = (size_t)(2 * c->M + 1) * sizeof(float);
+    for (long long t = t0; t < t0 + steps; ++t) {
+        a.t = t;
+        a.first = t == t0;
+        if (eager) k_eager_token<<<(unsigned)c->G, threads, smem, c->stream>>>(a);
+        else k_lazy_token<<<(unsigned)c->G, threads, smem, c->stream>>>(a);
+    }
+    CK(cudaGetLastError());
+    c->launches += steps;
+    c->last_trace = nullptr;
+    return FI_OK;
+}
+
 int run(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed) {
+    if (c->path >= FI_PATH_LAZY) return run_baseline(c, t0, steps, x, out, closed);
     const bool window = c->path == FI_PATH_WINDOW && c->W > 0;
     c->enq_launches = 0;
     if (!c->graphs || !window) {
@@ -1099,9 +1130,12 @@ int fi_set_stream(fi_ctx* ctx, void* stream) {
 int fi_set_path(fi_ctx* ctx, int path) {
     int rc = check_ctx(ctx);
     if (rc) return rc;
-    if (path != FI_PATH_WINDOW && path != FI_PATH_TOKEN) return set_err(FI_EINVAL, "unknown path %d", path);
+    if (path < FI_PATH_WINDOW || path > FI_PATH_EAGER) return set_err(FI_EINVAL, "unknown path %d", path);
     if (path == FI_PATH_WINDOW && ctx->W == 0)
         return set_err(FI_EINVAL, "window path unavailable for this shape (shared memory)");
+    const bool base_new = path >= FI_PATH_LAZY, base_old = ctx->path >= FI_PATH_LAZY;
+    if (path != ctx->path && ctx->t != 0 && (base_new || base_old))
+        return set_err(FI_EINVAL, "the lazy and eager paths keep their own state: switch to or from them at t = 0");
     ctx->path = path;
     return FI_OK;
 }

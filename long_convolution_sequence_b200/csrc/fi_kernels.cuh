@@ -1275,3 +1275,6 @@ __global__ void k_read_layer(const float* __restrict__ act, long long L, long lo
 
 // cluster FFT tau (blocks beyond one CTA's shared memory)
 #include "fi_cluster.cuh"
+
+// the Lazy and Eager baselines
+#include "fi_baselines.cuh"
