@@ -958,12 +958,15 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
             const long long g = (long long)(i / nch) * D + c0 + (i % nch);
             cp_async16(sm + (l * CPB + i) * P + 4 * c4, a.act + ((long long)l * G + g) * L + kW + 4 * c4);
         }
-        // the zero row before the first row and the padding after every row
+        // the zero row before the first row and the padding after every row (16-byte
+        // stores: rows start on 16-byte boundaries, W and kWinPad are multiples of 4)
+        static_assert(W % 4 == 0 && kWinPad % 4 == 0, "16-byte padding stores");
         for (int e = tid; e < P; e += NT) sm[e - P] = 0.f;
         const int nrows = dup0 / P + M * CPB;
-        for (int e = tid; e < nrows * kWinPad; e += NT) {
-            const int r = e / kWinPad;
-            sm[r * P + W + (e - r * kWinPad)] = 0.f;
+        for (int r = tid; r < nrows; r += NT) {
+            float4* pr = reinterpret_cast<float4*>(sm + r * P + W);
+#pragma unroll
+            for (int k = 0; k < kWinPad / 4; ++k) pr[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         cp_async_commit();
         cp_async_wait_all();
@@ -984,11 +987,15 @@ __global__ void __launch_bounds__(kWinThreads, 1) k_window(WinArgs a) {
         }
         __syncthreads();
         // shifted copies of the input rows (only positions already final are ever
-        // read); entry 0 stands for position -1 and is zero
-        for (int e = tid; e < M * ncb * W; e += NT) {
-            const int row = e / W, x = e - row * W;
-            const int l = row / ncb, i = row - l * ncb;
-            dup[(l * CPB + i) * P + x] = x == 0 ? 0.f : slot[(l * CPB + i) * P + x - 1];
+        // read); entry 0 stands for position -1 and is zero.  Every row l * CPB + i of
+        // layers 0..M-1 is copied, the unused ones (i >= ncb) too: thread -> column
+        // x = tid % W, rows advance by NT / W
+        {
+            constexpr int RS = NT / W;
+            const int x = tid & (W - 1);
+            if (tid < RS * W)
+                for (int r = tid / W; r < M * CPB; r += RS)
+                    dup[r * P + x] = x == 0 ? 0.f : slot[r * P + x - 1];
         }
         __syncthreads();
     }
