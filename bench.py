@@ -225,7 +225,12 @@ def main():
     ap.add_argument("--baseline", choices=("lazy", "eager"),
                     help="time the pages' Lazy or Eager baseline on this device next to the tiled path "
                          "(default workload: short)")
+    ap.add_argument("--prefill", default=None,
+                    help="comma-separated prompt lengths: time fi_prefill against the online "
+                         "teacher-forced path over the same prompt (headline stack)")
     args = ap.parse_args()
+    if args.prefill:
+        return bench_prefill(args)
     if args.sweep:
         return bench_sweep(args)
     if args.baseline:
@@ -550,6 +555,48 @@ def bench_baseline(args):
             "finite": finite, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl, "layers": M, "B": B, "D": D, "L": L}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_prefill(args):
+    """Prompt prefill (fi_prefill: one FFT convolution per layer) against the online
+    teacher-forced path (fi_forward) over the same prompt, on the workload's stack; CUDA
+    events, 2 warm-ups and 3 timed runs each; one JSON line per prompt length."""
+    import torch
+    import long_convolution_sequence_b200 as fi
+    from long_convolution_sequence_b200 import synth
+    M, B, D, L = WORKLOADS[args.workload]
+    h = synth.filters(M, D, L, seed=0)
+    ctx = fi.FlashInference(M, B, D, L, h)
+    for p in [int(v) for v in args.prefill.split(",")]:
+        x = torch.from_numpy(synth.inputs(p, B, D, seed=0)).cuda()
+        y = torch.empty((p, B, D), device="cuda")
+
+        def timed(fn, n=3):
+            for _ in range(2):
+                ctx.reset()
+                fn()
+            torch.cuda.synchronize()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            tot = 0.0
+            for _ in range(n):
+                ctx.reset()
+                ev0.record()
+                fn()
+                ev1.record()
+                torch.cuda.synchronize()
+                tot += ev0.elapsed_time(ev1)
+            return tot / n
+
+        pre_ms = timed(lambda: ctx.prefill(x, p, y))
+        y_pre = y.clone()
+        on_ms = timed(lambda: ctx.forward(x, p, y))
+        err = float((y_pre - y).abs().max() / y.pow(2).mean().sqrt())
+        print(json.dumps({"metric": "prompt tokens/s", "prompt": p, "prefill_ms": round(pre_ms, 3),
+                          "online_ms": round(on_ms, 3), "speedup": round(on_ms / pre_ms, 2),
+                          "prefill_value": round(B * p / (pre_ms / 1e3), 1), "max_err_over_rms": err,
+                          "config": {"workload": args.workload, "layers": M, "B": B, "D": D, "L": L}}), flush=True)
+    ctx.close()
     return 0
 
 

@@ -24,6 +24,8 @@
  *   [Base]  section "Kern-Algorithmus: Relaxierte Polynominterpolation", part 1 (the
  *           Lazy and Eager evaluations) and "Vergleichsmethoden" (their parallel
  *           versions as the baselines)
+ *   [Pre]   the rebuttal's note on prefill (appendix A.3 as cited there): the prompt
+ *           is taken eagerly before the autoregressive stage
  *   [Lem1]  section "Beitrags-Aggregations-Definition", Lemma 1:
  *           tau(y,[l,r],rho,[l',r'])_t = sum_{i=l}^{r} y_i rho_{t-i}
  *
@@ -137,6 +139,21 @@ int fi_generate(fi_ctx *ctx, const float *x0, int steps, float *out);
 /* Teacher-forced run over `steps` tokens (the windowed form of fi_step):
  * x [steps][B][D] are tokens t .. t+steps-1, y [steps][B][D] receives y^M. */
 int fi_forward(fi_ctx *ctx, const float *x, int steps, float *y);
+
+/* Prompt prefill ([Pre]): the p-token prompt x [p][B][D] (teacher-forced tokens
+ * 0..p-1) folded in layer by layer with one FFT convolution per layer (the block tau
+ * of [Lem1] with U = the power of two >= p and the taps shifted by U, so that only
+ * lags 0..t reach position t) instead of p online steps; y [p][B][D] receives y^M of
+ * the prompt positions.  Afterwards t = p and the buffers hold exactly the tiled
+ * paths' state (every block released up to p applied, activations final below p),
+ * so fi_generate / fi_forward / fi_step continue the sequence.  Needs t = 0 (after
+ * fi_create or fi_reset) and a tiled path (FI_PATH_WINDOW or FI_PATH_TOKEN), else
+ * FI_EINVAL; 1 <= p <= L.  Prompts shorter than 8 tokens take the online path.
+ * The context keeps about 4 * B * D * (4U + M U / 2) bytes of device scratch from the
+ * first prefill of that size on (FI_ENOMEM if it cannot get it), freed with the
+ * context.  Asynchronous on the context's stream like fi_forward; with host buffers
+ * it synchronises before returning. */
+int fi_prefill(fi_ctx *ctx, const float *x, int p, float *y);
 
 /* Rewind to t = 0 for a new sequence.  O(1): stale buffer contents are never read
  * (the first block written onto any position overwrites instead of accumulating). */

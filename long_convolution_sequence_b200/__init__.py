@@ -51,6 +51,7 @@ SIGNATURES = {
     "fi_step": (_I, [_P, _P, _P]),
     "fi_generate": (_I, [_P, _P, _I, _P]),
     "fi_forward": (_I, [_P, _P, _I, _P]),
+    "fi_prefill": (_I, [_P, _P, _I, _P]),
     "fi_reset": (_I, [_P]),
     "fi_read_layer": (_I, [_P, _I, _I, _I, _P]),
     "fi_set_stream": (_I, [_P, _P]),
@@ -152,6 +153,10 @@ class FlashInference:
 
     def forward(self, x, steps: int, y):
         _check(get_lib().fi_forward(self._h, _ptr(x), steps, _ptr(y)))
+
+    def prefill(self, x, p: int, y):
+        """Fold a p-token prompt in with one FFT convolution per layer: see fi_prefill."""
+        _check(get_lib().fi_prefill(self._h, _ptr(x), p, _ptr(y)))
 
     def reset(self):
         _check(get_lib().fi_reset(self._h))

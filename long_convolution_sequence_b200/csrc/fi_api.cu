@@ -115,6 +115,8 @@ struct fi_ctx {
     size_t sx_n = 0;
     float* sy = nullptr;  // staging for host outputs
     size_t sy_n = 0;
+    float* pre = nullptr;  // prompt-prefill scratch, grown on demand
+    size_t pre_n = 0;
     std::map<GraphKey, GraphEntry> gcache;
     std::vector<GraphKey> gorder;
     size_t bytes = 0;
@@ -520,8 +522,9 @@ TileArgs stack_tile_args(const fi_ctx* c, long long n) {
 
 // The gray blocks of every layer released after the n-th token, one launch
 // (section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)").
-int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st, int pdl = 0) {
+int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st, int pdl = 0, int force_acc = 0) {
     TileArgs a = stack_tile_args(c, n);
+    if (force_acc) a.overwrite = 0;
     const int q = ctz64(n);
     const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
                     : (q <= fused_qmax() ? FI_K_BLOCK_FFT : FI_K_BLOCK_CLUSTER);
@@ -948,6 +951,7 @@ void free_ctx(fi_ctx* c) {
     for (int q = 0; q < 32; ++q) cudaFree(c->spec[q]);
     cudaFree(c->sx);
     cudaFree(c->sy);
+    cudaFree(c->pre);
     for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
     if (c->cap) cudaStreamDestroy(c->cap);
     c->magic = 0;
@@ -986,6 +990,82 @@ int create_impl(fi_ctx* c, const float* filters) {
 }  // namespace
 
 // ====================================================================== C-ABI
+// Prompt prefill (x, y device pointers): the prompt's activations layer by layer, one
+// FFT convolution per layer (U = the power of two >= p), then the state the tiled path
+// expects at t = p: the running sum of every position >= p holds the blocks released
+// up to p.  Those are the blocks n <= p whose outputs reach past p (n + lowbit(n) > p);
+// the largest power of two n0 <= p is the first and widest, its outputs [n0, 2 n0)
+// cover every other's.  They are replayed through the ordinary block launches onto
+// zeroed positions [p, 2 n0), accumulating, in decreasing n: a block writes only at
+// positions >= its own n, so no replayed block clobbers the inputs of one still to
+// come.  Their outputs below p, already final activations, are saved before and
+// restored after.
+int prefill_impl(fi_ctx* c, const float* x, int p, float* y) {
+    const long long G = c->G, L = c->L;
+    const int M = c->M;
+    int U = 1 << kFftQMin;
+    while (U < p) U <<= 1;
+    const int q = ctz64(U);
+    cudaStream_t st = c->stream;
+    // scratch (kept by the context): blocks [G][U], out [G][U], taps [G][2U], spectra
+    // [G][U + 2] complex, the saved activations [M][G][p - n0] (p - n0 < U / 2)
+    const size_t nb = (size_t)G * U, nspec = (size_t)G * fused_stride(U);
+    const size_t need = 4 * nb + 2 * nspec + (size_t)M * G * (U / 2);
+    int rc;
+    if ((rc = ensure_stage(c, &c->pre, &c->pre_n, need))) return rc;
+    float* blocks = c->pre;
+    float* out = blocks + nb;
+    float* taps = out + nb;
+    float2* spec = reinterpret_cast<float2*>(taps + 2 * nb);  // 8-byte aligned: 4 nb floats before it
+    float* saved_area = reinterpret_cast<float*>(spec + nspec);
+    const int grid = 4 * c->nsm, nt = 256;
+    k_prefill_input<<<grid, nt, 0, st>>>(x, G, L, p, c->act);
+    long long nl = 1;
+    for (int l = 1; l <= M; ++l) {
+        k_prefill_gather<<<grid, nt, 0, st>>>(c->act, l - 1, G, L, p, U, blocks);
+        k_prefill_taps<<<grid, nt, 0, st>>>(c->h, l, c->D, G, L, U, taps);
+        if ((rc = make_spectra(q, taps, 2 * U, (int)G, spec, c->tw, st))) return rc;
+        TileArgs a;
+        memset(&a, 0, sizeof(a));
+        a.flat = 1;
+        a.fin = blocks;
+        a.fout = out;
+        a.ftaps = taps;
+        a.ldt = 2 * U;
+        a.U = U;
+        a.count = (int)G;
+        a.overwrite = 1;
+        a.tw = c->tw;
+        a.twlog = kTwLog;
+        a.spec = spec;
+        a.spec_stride = fused_stride(U);
+        if ((rc = launch_fft(q, a, st))) return rc;
+        k_prefill_scatter<<<grid, nt, 0, st>>>(out, l, G, L, p, U, c->act, l == M ? y : nullptr);
+        nl += 5;
+    }
+    CK(cudaGetLastError());
+    long long n0 = 1;
+    while (2 * n0 <= p) n0 <<= 1;  // the first open block: the largest power of two <= p
+    float* saved = nullptr;
+    if (n0 < p) {
+        saved = saved_area;
+        k_prefill_rows<<<grid, nt, 0, st>>>(c->act, saved, M, G, L, (int)n0, p, 1);
+    }
+    const long long zend = std::min<long long>(2 * n0, L);
+    if (zend > p)
+        CK(cudaMemset2DAsync(c->act + G * L + p, sizeof(float) * L, 0, sizeof(float) * (zend - p), (size_t)M * G, st));
+    for (long long n = std::min<long long>(p, L - 1); n >= n0; --n) {
+        if (n + lowbit(n) <= p) continue;
+        if ((rc = launch_block(c, n, tau_of(c, ctz64(n)), st, 0, 1))) return rc;
+        ++nl;
+    }
+    if (saved) k_prefill_rows<<<grid, nt, 0, st>>>(c->act, saved, M, G, L, (int)n0, p, 0);
+    CK(cudaGetLastError());
+    c->launches += nl;
+    c->last_trace = nullptr;
+    return FI_OK;
+}
+
 extern "C" {
 
 const char* fi_last_error(void) { return g_err; }
@@ -1095,6 +1175,36 @@ int fi_step(fi_ctx* ctx, const float* x_t, float* y_t) {
 int fi_generate(fi_ctx* ctx, const float* x0, int steps, float* out) { return run_call(ctx, x0, steps, out, 1); }
 
 int fi_forward(fi_ctx* ctx, const float* x, int steps, float* y) { return run_call(ctx, x, steps, y, 0); }
+
+int fi_prefill(fi_ctx* ctx, const float* x, int p, float* y) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (ctx->t != 0) return set_err(FI_EINVAL, "fi_prefill starts a sequence: call it at t = 0 (fi_reset)");
+    if (p < 1 || p > ctx->L) return set_err(FI_EINVAL, "fi_prefill: need 1 <= p <= L = %d", ctx->L);
+    if (!x || !y) return set_err(FI_EINVAL, "fi_prefill: x and y must be non-NULL");
+    if (ctx->path >= FI_PATH_LAZY) return set_err(FI_EINVAL, "fi_prefill serves the tiled paths only");
+    if (p < (1 << kFftQMin)) return run_call(ctx, x, p, y, 0);  // a few tokens: the online path
+    const long long G = ctx->G;
+    const float* xd = x;
+    float* yd = y;
+    const bool x_host = !is_device_ptr(x), y_host = !is_device_ptr(y);
+    if (x_host) {
+        if ((rc = ensure_stage(ctx, &ctx->sx, &ctx->sx_n, (size_t)G * p))) return rc;
+        CK(cudaMemcpyAsync(ctx->sx, x, sizeof(float) * G * p, cudaMemcpyHostToDevice, ctx->stream));
+        xd = ctx->sx;
+    }
+    if (y_host) {
+        if ((rc = ensure_stage(ctx, &ctx->sy, &ctx->sy_n, (size_t)G * p))) return rc;
+        yd = ctx->sy;
+    }
+    if ((rc = prefill_impl(ctx, xd, p, yd))) return rc;
+    ctx->t = p;
+    if (y_host) {
+        CK(cudaMemcpyAsync(y, yd, sizeof(float) * G * p, cudaMemcpyDeviceToHost, ctx->stream));
+        CK(cudaStreamSynchronize(ctx->stream));
+    }
+    return FI_OK;
+}
 
 int fi_read_layer(fi_ctx* ctx, int layer, int t0, int t1, float* dst) {
     int rc = check_ctx(ctx);

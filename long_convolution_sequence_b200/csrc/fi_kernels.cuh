@@ -1285,3 +1285,6 @@ __global__ void k_read_layer(const float* __restrict__ act, long long L, long lo
 
 // the Lazy and Eager baselines
 #include "fi_baselines.cuh"
+
+// the prompt prefill's element-wise kernels
+#include "fi_prefill.cuh"
