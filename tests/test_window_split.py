@@ -2,10 +2,11 @@
 
 The window kernel splits the relaxed tiling's in-window blocks (section
 "Kachelung-Strategie (Algorithmus 1)" of the Flash Inference summary) between three
-roles: the chain lanes add lags 1 and 2 of the current position, the helper pairs add
-the rows of every lag >= 3, and a launch that stops inside the window completes the
-blocks it released.  This restates those decisions (the lag-2 parity rule, the helper
-rows' cover ranges, the completion step) exactly as the kernel takes them and checks,
+roles: the chain lanes add lags 1 .. K-1 of the current position (K = 3), the helper
+pairs add the rows of every lag >= K, and a launch that stops inside the window completes the
+blocks it released.  This restates those decisions (a chain lag is added when its
+block was released after the launch began, by the closed forms of those blocks; the
+helper rows' cover ranges; the completion step) as the kernel takes them and checks,
 against brute force over the tiling, that after every launch of every split of a
 window each pair of a block released so far has been applied exactly once and no
 other pair has."""
@@ -42,26 +43,29 @@ def cover_range(T, s0, hi):
     return lo, top
 
 
-def lag2_pending(s, s0):
-    # the block holding (s - 2, s) is n = s - 1 for odd s, else n = s
-    return s > s0 + 1 if s & 1 else s > s0
+def lag_block(s, d):
+    # the block holding the pair (s - d, s), d = 1, 2, 3, in closed form
+    if d == 1:
+        return s
+    if d == 2:
+        return s - 1 if s & 1 else s
+    return (s, s - 1, s - 2, s - 1)[s & 3]
 
 
-def launch(W, s0, s1):
+def launch(W, s0, s1, K):
     added = []
     for s in range(s0, s1):
-        if s > s0:
-            added.append((s - 1, s))
-        if lag2_pending(s, s0):
-            added.append((s - 2, s))
+        for d in range(1, K):
+            if s - d >= 0 and lag_block(s, d) > s0:
+                added.append((s - d, s))
         T = s + 1
         if T < W:
             lo = 0 if s0 == 0 else cover_range(T, s0, T)[0]
-            added += [(j, T) for j in range(lo, T - 2)]  # lags >= 3
+            added += [(j, T) for j in range(lo, T - K + 1)]  # lags >= K
     if s0 < s1 < W:
-        added.append((s1 - 1, s1))
-        if (s1 & 1) == 0 or s1 > s0 + 1:
-            added.append((s1 - 2, s1))
+        for d in range(1, K):
+            if s1 - d >= 0 and lag_block(s1, d) > s0:
+                added.append((s1 - d, s1))
         for T in range(s1 + 1, W):
             lo, top = cover_range(T, s0, s1)
             if lo >= 0:
@@ -74,11 +78,11 @@ def blocks(W):
     return {(j, p): block_of(j, p) for p in range(W) for j in range(p)}
 
 
-def check(W, splits):
+def check(W, splits, K):
     applied = {}
     pts = [0] + list(splits) + [W]
     for s0, s1 in zip(pts[:-1], pts[1:]):
-        for pr in launch(W, s0, s1):
+        for pr in launch(W, s0, s1, K):
             assert 0 <= pr[0] < pr[1] < W, pr
             applied[pr] = applied.get(pr, 0) + 1
         want = {pr for pr, n in blocks(W).items() if n <= s1}
@@ -86,20 +90,29 @@ def check(W, splits):
         assert set(applied) == want, (splits, s0, s1)
 
 
+def test_lag_blocks_closed_forms():
+    for s in range(3, 2048):
+        for d in (1, 2, 3):
+            assert lag_block(s, d) == block_of(s - d, s)
+
+
+@pytest.mark.parametrize("K", [3])
 @pytest.mark.parametrize("W", [32, 64])
-def test_whole_window_and_every_single_split(W):
-    check(W, [])
+def test_whole_window_and_every_single_split(W, K):
+    check(W, [], K)
     for a in range(1, W):
-        check(W, [a])
+        check(W, [a], K)
 
 
-def test_every_two_way_split():
+@pytest.mark.parametrize("K", [3])
+def test_every_two_way_split(K):
     W = 32
     for a, b in itertools.combinations(range(1, W), 2):
-        check(W, [a, b])
+        check(W, [a, b], K)
 
 
-def test_random_splits_of_the_128_window():
+@pytest.mark.parametrize("K", [3])
+def test_random_splits_of_the_128_window(K):
     rng = random.Random(7)
     for _ in range(40):
-        check(128, sorted(rng.sample(range(1, 128), rng.randint(1, 10))))
+        check(128, sorted(rng.sample(range(1, 128), rng.randint(1, 10))), K)
