@@ -63,9 +63,11 @@ def test_calls_on_null_context_report_state_error(lib):
     assert lib.fi_step(None, p, p) == fi.FI_ESTATE
     assert lib.fi_generate(None, p, 1, p) == fi.FI_ESTATE
     assert lib.fi_forward(None, p, 1, p) == fi.FI_ESTATE
+    assert lib.fi_prefill(None, p, 8, p) == fi.FI_ESTATE
     assert lib.fi_reset(None) == fi.FI_ESTATE
     assert lib.fi_read_layer(None, 0, 0, 0, p) == fi.FI_ESTATE
     assert lib.fi_set_path(None, 0) == fi.FI_ESTATE
+    assert lib.fi_set_path(None, fi.FI_PATH_LAZY) == fi.FI_ESTATE
     assert lib.fi_set_tau(None, 0, 1) == fi.FI_ESTATE
     assert lib.fi_get_info(None, ctypes.byref(fi.fi_info())) == fi.FI_ESTATE
     assert b"context" in lib.fi_last_error()
