@@ -169,6 +169,20 @@ def test_window_launch_of_several_waves(window):
     assert rel(y, ref["y_last"]) < TOL_TF
 
 
+def test_closed_loop_on_a_window_launch_of_several_waves(window):
+    # as above, two waves of 3-channel CTAs, now in the closed loop
+    M, B, D, L = 18, 4, 512, 512
+    window(64)
+    h = synth.filters(M, D, L, seed=5)
+    x0 = synth.start_token(B, D, seed=5)
+    ref = oracle.stack(h, x0, T=L, closed_loop=True, want=("y_last",))["y_last"]
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        assert ctx.info().window == 64
+        out = np.empty((L, B, D), np.float32)
+        ctx.generate(x0, L, out)
+    assert rel(out, ref) < TOL_CL
+
+
 @pytest.mark.parametrize("M,B,D,L,W", [(1, 1, 16, 1024, None), (3, 2, 6, 4096, 64), (18, 1, 8, 4096, None)])
 def test_closed_loop_matches_oracle(M, B, D, L, W, window):
     window(W)

@@ -48,6 +48,19 @@ def test_prefill_then_forward_matches_the_oracle(stack, p, path):
 
 
 @pytest.mark.gpu
+def test_prefill_of_the_18_layer_stack_with_a_batch():
+    M, B, D, L, p = 18, 2, 5, 2048, 777
+    h = synth.filters(M, D, L, seed=14)
+    x = synth.inputs(L, B, D, seed=14)
+    ref = oracle.stack(h, x, want=("y_last",))["y_last"]
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        y = np.empty((L, B, D), np.float32)
+        ctx.prefill(np.ascontiguousarray(x[:p]), p, y[:p])
+        ctx.forward(np.ascontiguousarray(x[p:]), L - p, y[p:])
+    assert rel(y, ref) < TOL_TF
+
+
+@pytest.mark.gpu
 def test_short_prompt_takes_the_online_path(stack):
     M, B, D, L, h, x, ref = stack
     with fi.FlashInference(M, B, D, L, h) as ctx:
