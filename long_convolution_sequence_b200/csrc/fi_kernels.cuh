@@ -259,74 +259,10 @@ __device__ __forceinline__ void unpack_pair(float2 Zk, float2 Zn, float2 Wk, flo
     if (k0) Xn = make_float2(E.x - O.x, E.y - O.y);      // X[N] = E[0] - O[0]
     else Xn = cadd(conjf2(E), cmul(Wnk, conjf2(O)));    // E[N-k] = conj E[k], same for O
 }
-// Inverse of the packing: from Y[k] and Y[N-k] of a real 2N-point signal y, the
-// values Z'[k] = E'[k] + i O'[k] with E'[k] = (Y[k] + conj Y[N-k]) / 2 and
-// O'[k] = (Y[k] - conj Y[N-k]) W^{-k} / 2, so that IDFT_N(Z')[m] = y[2m] + i y[2m+1].
-__device__ __forceinline__ float2 repack(float2 Yk, float2 Yn, float2 Wk) {
-    float2 E = make_float2(0.5f * (Yk.x + Yn.x), 0.5f * (Yk.y - Yn.y));
-    float2 Q = make_float2(0.5f * (Yk.x - Yn.x), 0.5f * (Yk.y + Yn.y));
-    float2 O = cmul(Q, conjf2(Wk));
-    return make_float2(E.x - O.y, E.y + O.x);  // E + i O
-}
-
 // Twiddle e^{-2 pi i k / 2N} from the table e^{-2 pi i m / 2^twlog}.
 template <int LOGN>
 __device__ __forceinline__ float2 tw2n(const float2* __restrict__ tw, int twlog, int k) {
     return __ldg(&tw[k << (twlog - LOGN - 1)]);
-}
-
-// After the forward FFT of a packed, half-zero block (X = Z), form Y = X (.) H and
-// store conj of the repacked Z' so that a second forward FFT gives N conj(z').
-template <int LOGN, int NT>
-__device__ __forceinline__ void spectral_multiply(float2* X, const float2* __restrict__ H,
-                                                  const float2* __restrict__ tw, int twlog) {
-    constexpr int N = 1 << LOGN;
-    for (int k = threadIdx.x; k <= N / 2; k += NT) {
-        const int kn = (N - k) & (N - 1);
-        float2 Zk = X[k], Zn = X[kn];
-        float2 Wk = tw2n<LOGN>(tw, twlog, k);
-        float2 Wnk = tw2n<LOGN>(tw, twlog, N - k);
-        float2 Xk, Xn;
-        unpack_pair(Zk, Zn, Wk, Wnk, k == 0, Xk, Xn);
-        float2 Yk = cmul(Xk, __ldg(&H[k]));
-        float2 Yn = cmul(Xn, __ldg(&H[N - k]));
-        float2 Zpk = repack(Yk, Yn, Wk);
-        X[k] = conjf2(Zpk);
-        if (k != 0 && kn != k) {
-            float2 Zpn = repack(Yn, Yk, Wnk);
-            X[kn] = conjf2(Zpn);
-        }
-    }
-    __syncthreads();
-}
-
-// Write outputs [U, 2U-1] of the circular convolution (U = N): after the second
-// forward FFT, F = N conj(z'), so y[2m] = Re F[m] / N and y[2m+1] = -Im F[m] / N.
-template <int LOGN, int NT>
-__device__ __forceinline__ void store_upper_half(const float2* X, float* out, int overwrite) {
-    constexpr int N = 1 << LOGN;
-    const float inv = 1.0f / (float)N;
-    float2* o2 = reinterpret_cast<float2*>(out);
-    for (int m = N / 2 + threadIdx.x; m < N; m += NT) {
-        float2 F = X[m];
-        float2 v = make_float2(F.x * inv, -F.y * inv);
-        const int q = m - N / 2;
-        if (overwrite) o2[q] = v;
-        else {
-            float2 old = o2[q];
-            o2[q] = make_float2(old.x + v.x, old.y + v.y);
-        }
-    }
-}
-
-// Load a block of U = N floats as N/2 packed complex values followed by N/2 zeros.
-template <int LOGN, int NT>
-__device__ __forceinline__ void load_half_zero(float2* X, const float* in) {
-    constexpr int N = 1 << LOGN;
-    const float2* i2 = reinterpret_cast<const float2*>(in);
-    for (int m = threadIdx.x; m < N / 2; m += NT) X[m] = i2[m];
-    for (int m = N / 2 + threadIdx.x; m < N; m += NT) X[m] = make_float2(0.f, 0.f);
-    __syncthreads();
 }
 
 // ----------------------------------------------------------------- fused FFT tau
@@ -739,43 +675,6 @@ __device__ __forceinline__ float dot_pair(const float* in, const float* tp, int 
             a2 = fmaf(x[u + 2], y[u + 2], a2);
             a3 = fmaf(x[u + 3], y[u + 3], a3);
         }
-    }
-    return (a0 + a1) + (a2 + a3);
-}
-
-// The main-loop row of a helper lane's own item with its taps in registers: lane
-// `part` of the pair takes the lags d = 2 + part + 2m, m < nm_me, and adds
-// in[T - d] * tap[d] with tr[m] = tap[2 + part + 2m]; pin = in + T - 2 - part, so term
-// m reads pin[-2m].  nm_both (<= nm_me <= nm_both + 1) terms are valid for both lanes
-// of the pair.  Terms go in blocks of 8 whose loads are issued before their
-// multiply-adds; the block holding the pair's last term is masked per term.  Every
-// index into tr is a compile-time constant, so the taps stay in registers.
-template <int NTR>
-__device__ __forceinline__ float dot_lags(const float* pin, const float (&tr)[NTR], int nm_both, int nm_me) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-    for (int b = 0; b < NTR; b += 8) {
-        if (b >= nm_me) break;
-        float x[8];
-        if (b + 8 <= nm_both) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) x[u] = pin[-2 * (b + u)];
-        } else {
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const bool ok = b + u < nm_me;
-                const float v = pin[ok ? -2 * (b + u) : 0];
-                x[u] = ok ? v : 0.f;
-            }
-        }
-        a0 = fmaf(x[0], tr[b + 0], a0);
-        a1 = fmaf(x[1], tr[b + 1], a1);
-        a2 = fmaf(x[2], tr[b + 2], a2);
-        a3 = fmaf(x[3], tr[b + 3], a3);
-        a0 = fmaf(x[4], tr[b + 4], a0);
-        a1 = fmaf(x[5], tr[b + 5], a1);
-        a2 = fmaf(x[6], tr[b + 6], a2);
-        a3 = fmaf(x[7], tr[b + 7], a3);
     }
     return (a0 + a1) + (a2 + a3);
 }
