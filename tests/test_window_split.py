@@ -116,3 +116,58 @@ def test_random_splits_of_the_128_window(K):
     rng = random.Random(7)
     for _ in range(40):
         check(128, sorted(rng.sample(range(1, 128), rng.randint(1, 10))), K)
+
+
+# ---------------------------------------------------------------- helper-row reads
+# The helper pair of one (layer, chain) item computes row T over lags 3 .. T - lo in
+# lag pairs (3 + 2k, 4 + 2k), pair k = part + 2m on lane `part`, one 8-byte load per
+# pair at positions (T - 4 - 2k, T - 3 - 2k).  Rows whose blocks start at window
+# position 0 run whole blocks of 8 pairs and rely on 36 zero floats before each row;
+# the others mask per term.  These restate the kernel's index arithmetic and check
+# that every lag is taken exactly once and no read leaves the row or its padding.
+PAD = 36
+
+
+def helper_terms(T, lo, padded, W):
+    dmax = T - lo
+    K = (dmax - 1) >> 1
+    terms, low = [], 0
+    for part in (0, 1):
+        if padded:
+            nblk = (((K + 1) >> 1) + 7) >> 3
+            assert 8 * nblk <= ((W - 2) // 4 + 7) // 8 * 8  # register tap pairs
+            for m in range(8 * nblk):
+                k = part + 2 * m
+                for d, pos in ((4 + 2 * k, T - 4 - 2 * k), (3 + 2 * k, T - 3 - 2 * k)):
+                    low = min(low, pos)
+                    if pos >= 0 and d < W:
+                        terms.append((d, pos))
+                    else:  # a zero from the padding, or a zero tap past the window
+                        assert pos < 0 or d >= W
+        else:
+            nm_me = (K - part + 1) >> 1
+            last_half = (dmax & 1) == 1 and ((K - 1) & 1) == part
+            for m in range(nm_me):
+                k = part + 2 * m
+                if not (last_half and m == nm_me - 1):
+                    terms.append((4 + 2 * k, T - 4 - 2 * k))
+                terms.append((3 + 2 * k, T - 3 - 2 * k))
+    if not padded:
+        low = min((p for _, p in terms), default=lo)
+    return terms, low
+
+
+@pytest.mark.parametrize("W", [32, 64, 128, 256])
+def test_helper_rows_take_every_lag_once_and_stay_in_bounds(W):
+    for T in range(1, W):
+        for lo in range(0, T):
+            for padded in ((True, False) if lo == 0 else (False,)):
+                terms, low = helper_terms(T, lo, padded, W)
+                assert sorted(d for d, _ in terms) == list(range(3, T - lo + 1)), (T, lo, padded)
+                assert all(T - d == p for d, p in terms)
+                if padded:
+                    assert low >= -31 and 31 < PAD, (T, low)
+                else:
+                    assert low >= lo, (T, lo, low)
+            # the 8-byte load of pair 0 is aligned in the row (T even) or its shifted copy
+            assert ((T - 4) % 2 == 0) == (T % 2 == 0)
