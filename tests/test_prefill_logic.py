@@ -63,6 +63,8 @@ def test_open_blocks_rebuild_the_tiled_state_after_a_prompt(L):
         if blocks:
             n0 = 1 << (p.bit_length() - 1)
             assert min(blocks) == n0
+            # every replayed block writes inside [n0, 2 n0), so the activations it
+            # overwrites lie in [n0, p)
             assert all(n0 <= n and n + lowbit(n) <= 2 * n0 for n in blocks)
             # decreasing n: no replayed block writes a position that a block replayed
             # after it (smaller n) reads
@@ -72,5 +74,3 @@ def test_open_blocks_rebuild_the_tiled_state_after_a_prompt(L):
                         writes = set(range(a, a + lowbit(a)))
                         reads = set(range(b - lowbit(b), b))
                         assert not writes & reads, (p, a, b)
-            # the activations the replay overwrites lie in [n0, p)
-            assert all(max(n, 0) >= n0 for n in blocks)
