@@ -432,20 +432,12 @@ def sweep_need_bytes(M, B, D, L):
 
 
 def sweep_filters(M, D, L, seed=0):
-    """Filters of the sweep drawn on the device with the same law as the headline's
-    (h[c, k] = N(0,1) exp(-a_c k) / sqrt(32), a_c ~ U(0.001, 0.05), independent per
-    layer), from torch's seeded CUDA generator: the 2^18-tap filters of the largest
+    """Filters of the sweep drawn on the device (synth.device_filters: the headline's
+    law, h[c, k] = N(0,1) exp(-a_c k) / sqrt(32), a_c ~ U(0.001, 0.05), independent per
+    layer, from torch's seeded CUDA generator): the 2^18-tap filters of the largest
     points would take minutes on the host."""
-    import torch
-    h = torch.empty((M, D, L), device="cuda", dtype=torch.float32)
-    k = torch.arange(L, device="cuda", dtype=torch.float32)
-    for l in range(M):
-        g = torch.Generator(device="cuda")
-        g.manual_seed(1_000_003 * seed + l)
-        a = torch.empty(D, device="cuda").uniform_(0.001, 0.05, generator=g)
-        h[l].normal_(generator=g)
-        h[l] *= torch.exp(-a[:, None] * k[None, :]) / math.sqrt(32.0)
-    return h
+    from long_convolution_sequence_b200 import synth
+    return synth.device_filters(M, D, L, seed=seed)
 
 
 def bench_sweep(args):

@@ -223,7 +223,9 @@ int fi_tau(int impl, int U, int count, const float *blocks, const float *taps, i
  * GPU that loads the library holds until the process exits; large counts are
  * processed in chunks that fit it.  The first call on a device sets that device up
  * (looks up the array's device address and writes the twiddle table with a
- * synchronous copy), so make it before any stream capture.  Nothing in the array
+ * synchronous copy), so make it before any stream capture.  The set-up is tied to
+ * the device's context: after a cudaDeviceReset (or any teardown of the context) the
+ * library is loaded afresh with a new array, and the next call repeats the set-up.  Nothing in the array
  * needs to start at zero: each call writes every part it reads.  All calls share
  * the array, so calls that overlap on the GPU race (for example from two host
  * threads); calls are serialised on the legacy default stream and return after

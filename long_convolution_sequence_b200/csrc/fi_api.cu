@@ -588,14 +588,43 @@ constexpr int kNoAllocMaxDevices = 64;
 constexpr int kNoAllocQMax = 16;  // largest block (U = 65536) the fixed array serves
 std::mutex g_noalloc_mu;
 float2* g_noalloc_base[kNoAllocMaxDevices] = {};
+void* g_noalloc_ctx[kNoAllocMaxDevices] = {};  // context the set-up was made in
 
-// Once per device, with that device current: resolve the array's device address
-// (the host-side symbol is only a stand-in) and store the twiddle table in it.
+// The calling thread's current context (the driver's handle), looked up through the
+// runtime's driver entry point so that the library needs no link against libcuda.
+// A device reset or a context teardown gives the device a new context, in which the
+// module (and the fixed array) is loaded afresh: the cached address and the twiddle
+// table written into the old one no longer hold.
+int current_context(void** out) {
+    typedef int (*GetCurrent)(void**);
+    static GetCurrent fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) {
+            cudaGetLastError();
+            return set_err(FI_ECUDA, "fi_tau_fft_noalloc: cuCtxGetCurrent entry point unavailable");
+        }
+        fn = (GetCurrent)p;
+    }
+    *out = nullptr;
+    if (fn(out) != 0 || !*out) return set_err(FI_ECUDA, "fi_tau_fft_noalloc: no current CUDA context");
+    return FI_OK;
+}
+
+// Once per device and context, with that device current: resolve the array's device
+// address (the host-side symbol is only a stand-in) and store the twiddle table in it.
 int noalloc_setup(int dev, float2** base) {
     if (dev < 0 || dev >= kNoAllocMaxDevices)
         return set_err(FI_EINVAL, "fi_tau_fft_noalloc: device ordinal %d above %d", dev, kNoAllocMaxDevices - 1);
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_base[dev]) {
+    CK(cudaSetDevice(dev));  // makes the device's primary context current (creating it if needed)
+    void* ctx = nullptr;
+    int rc = current_context(&ctx);
+    if (rc) return rc;
+    if (!g_noalloc_base[dev] || g_noalloc_ctx[dev] != ctx) {
+        g_noalloc_base[dev] = nullptr;
         void* p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p) {
@@ -614,6 +643,7 @@ int noalloc_setup(int dev, float2** base) {
             return set_err(FI_ECUDA, "fi_tau_fft_noalloc: twiddle upload failed: %s", cudaGetErrorString(e));
         }
         g_noalloc_base[dev] = (float2*)p;
+        g_noalloc_ctx[dev] = ctx;
     }
     *base = g_noalloc_base[dev];
     return FI_OK;
@@ -1007,10 +1037,12 @@ int prefill_impl(fi_ctx* c, const float* x, int p, float* y) {
     while (U < p) U <<= 1;
     const int q = ctz64(U);
     cudaStream_t st = c->stream;
+    long long n0 = 1;
+    while (2 * n0 <= p) n0 <<= 1;  // the first open block: the largest power of two <= p
     // scratch (kept by the context): blocks [G][U], out [G][U], taps [G][2U], spectra
-    // [G][U + 2] complex, the saved activations [M][G][p - n0] (p - n0 < U / 2)
+    // [G][U + 2] complex, the saved activations [M][G][p - n0]
     const size_t nb = (size_t)G * U, nspec = (size_t)G * fused_stride(U);
-    const size_t need = 4 * nb + 2 * nspec + (size_t)M * G * (U / 2);
+    const size_t need = 4 * nb + 2 * nspec + (size_t)M * G * (size_t)(p - n0);
     int rc;
     if ((rc = ensure_stage(c, &c->pre, &c->pre_n, need))) return rc;
     float* blocks = c->pre;
@@ -1044,8 +1076,6 @@ int prefill_impl(fi_ctx* c, const float* x, int p, float* y) {
         nl += 5;
     }
     CK(cudaGetLastError());
-    long long n0 = 1;
-    while (2 * n0 <= p) n0 <<= 1;  // the first open block: the largest power of two <= p
     float* saved = nullptr;
     if (n0 < p) {
         saved = saved_area;
@@ -1181,6 +1211,9 @@ int fi_prefill(fi_ctx* ctx, const float* x, int p, float* y) {
     if (rc) return rc;
     if (ctx->t != 0) return set_err(FI_EINVAL, "fi_prefill starts a sequence: call it at t = 0 (fi_reset)");
     if (p < 1 || p > ctx->L) return set_err(FI_EINVAL, "fi_prefill: need 1 <= p <= L = %d", ctx->L);
+    if (p > (1 << kFftQMax))
+        return set_err(FI_EINVAL, "fi_prefill: p = %d above %d, the longest prompt one FFT convolution serves",
+                       p, 1 << kFftQMax);
     if (!x || !y) return set_err(FI_EINVAL, "fi_prefill: x and y must be non-NULL");
     if (ctx->path >= FI_PATH_LAZY) return set_err(FI_EINVAL, "fi_prefill serves the tiled paths only");
     if (p < (1 << kFftQMin)) return run_call(ctx, x, p, y, 0);  // a few tokens: the online path

@@ -70,6 +70,55 @@ def filters(M: int, D: int, L: int, seed: int = 0, decay: bool = True,
     return h
 
 
+def filter_rows(M: int, D: int, L: int, chans, T: int, seed: int = 0, decay: bool = True) -> np.ndarray:
+    """float32 [M][len(chans)][T]: ``filters(M, D, L, seed)[:, chans, :T]`` without
+    materialising the whole array.  Each layer's stream is drawn in the same order
+    and the same chunks as ``filters`` (every chunk is drawn whole and the rows asked
+    for are kept), so the values are bit-identical."""
+    chans = [int(c) for c in chans]
+    out = np.empty((M, len(chans), T), np.float32)
+    k = np.arange(L, dtype=np.float64)
+    chunk = 64
+
+    def layer(l):
+        g = _rng(seed, 1, l)
+        a = g.uniform(A_LO, A_HI, size=D)
+        if not decay:
+            a[:] = 0.0
+        for c0 in range(0, D, chunk):
+            c1 = min(D, c0 + chunk)
+            z = g.standard_normal((c1 - c0, L))
+            for i, c in enumerate(chans):
+                if c0 <= c < c1:
+                    row = z[c - c0] * np.exp(-a[c] * k)
+                    row *= SCALE
+                    out[l, i] = row[:T]
+
+    import os
+    threads = min(M, max(1, len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(layer, range(M)))
+    return out
+
+
+def device_filters(M: int, D: int, L: int, seed: int = 0):
+    """float32 [M][D][L] torch CUDA tensor with the filter law of ``filters`` drawn on
+    the device by torch's seeded CUDA generator (per layer ``manual_seed(1000003 *
+    seed + l)``: ``a_c`` for all c, then the normals).  A different draw from
+    ``filters``; used where host generation of long filters would take minutes (the
+    configuration sweep).  Copy it to the host to give the oracle the same array."""
+    import torch
+    h = torch.empty((M, D, L), device="cuda", dtype=torch.float32)
+    k = torch.arange(L, device="cuda", dtype=torch.float32)
+    for l in range(M):
+        g = torch.Generator(device="cuda")
+        g.manual_seed(1_000_003 * seed + l)
+        a = torch.empty(D, device="cuda").uniform_(A_LO, A_HI, generator=g)
+        h[l].normal_(generator=g)
+        h[l] *= torch.exp(-a[:, None] * k[None, :]) * SCALE
+    return h
+
+
 def inputs(T: int, B: int, D: int, seed: int = 0) -> np.ndarray:
     """float32 [T][B][D] teacher-forced tokens, N(0,1)."""
     return _rng(seed, 2).standard_normal((T, B, D)).astype(np.float32)

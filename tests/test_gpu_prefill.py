@@ -117,3 +117,21 @@ def test_prefill_argument_errors(stack):
         ctx.set_path(fi.FI_PATH_LAZY)
         with pytest.raises(fi.FiError):  # the baselines have no prefill
             ctx.prefill(np.ascontiguousarray(x[:64]), 64, y[:64])
+
+
+@pytest.mark.gpu
+def test_prefill_beyond_the_largest_fft_is_rejected_before_any_work():
+    # L = 2^18 is a valid capacity, but one FFT convolution serves prompts of at most
+    # 2^17 tokens: a longer prompt must fail with FI_EINVAL and leave the context at t = 0
+    M, B, D, L = 1, 1, 2, 1 << 18
+    h = synth.filters(M, D, L, seed=9)
+    p = (1 << 17) + 1
+    x = synth.inputs(p, B, D, seed=9)
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        y = np.empty((p, B, D), np.float32)
+        with pytest.raises(fi.FiError) as e:
+            ctx.prefill(x, p, y)
+        assert e.value.code == fi.FI_EINVAL and "131072" in str(e.value)
+        assert ctx.info().t == 0
+        ctx.prefill(np.ascontiguousarray(x[: 1 << 17]), 1 << 17, y[: 1 << 17])  # the largest one works
+        assert ctx.info().t == 1 << 17

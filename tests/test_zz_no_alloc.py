@@ -5,7 +5,10 @@ another allocator (a framework's caching pool, a serving engine that claims most
 of HBM at start-up), or they cannot accept the device-wide synchronisation an
 allocation may cost.  For them the library offers one entry point whose
 temporaries live in a fixed array of device memory inside the library itself.
-This file checks it against fi_tau, the allocating entry point, through the C-ABI.
+This file checks it through the C-ABI against fi_tau, the allocating entry point,
+and against the CPU oracle's tau (the sum of Lemma 1, section
+"Beitrags-Aggregations-Definition" of the Flash Inference paper summary): every
+output for the small blocks, sampled outputs for the large ones.
 
 The file is named so that pytest collects it last: if it fails, a run that stops
 at the first failure has already run every other test.  It must pass both alone
@@ -19,12 +22,32 @@ import numpy as np
 import pytest
 
 import long_convolution_sequence_b200 as fi
+import oracle
 
 TOL = 1e-4  # max |err| / RMS, the tolerance of the other tau parity tests
 
 
 def rel(got, ref):
     return float(np.abs(got - ref).max() / math.sqrt(float(np.mean(ref.astype(np.float64) ** 2))))
+
+
+def oracle_tau(blocks, taps, rng, k=48):
+    """The oracle's tau: (rows, reference) with every row r for U <= 4096, else k
+    sampled rows per block (first, last and random), each by the plain sum
+    sum_j blocks[i][j] taps[i][U + r - j] (a causal convolution sample at t = U + r
+    of the block padded with zeros)."""
+    count, U = blocks.shape
+    if U <= 4096:
+        return np.arange(U), oracle.tau(blocks, taps)
+    rows = np.unique(np.concatenate([[0, 1, U // 2, U - 1], rng.integers(0, U, size=k)]))
+    ref = np.empty((count, rows.size))
+    for i in range(count):
+        y = np.zeros(2 * U, np.float32)
+        y[:U] = blocks[i]
+        h = np.ascontiguousarray(taps[i])
+        for j, r in enumerate(rows):
+            ref[i, j] = oracle.conv_at(U + int(r), h, y)
+    return rows, ref
 
 
 def test_noalloc_rejects_blocks_beyond_its_scratch():
@@ -51,8 +74,10 @@ def test_noalloc_matches_fi_tau_on_two_calls_in_a_row(U, count):
     torch = pytest.importorskip("torch")
     rng = np.random.default_rng(1000 + U)
     for call in range(2):
-        blocks = torch.from_numpy(rng.standard_normal((count, U)).astype(np.float32)).cuda()
-        taps = torch.from_numpy(rng.standard_normal((count, 2 * U + 2)).astype(np.float32)).cuda()
+        blocks_h = rng.standard_normal((count, U)).astype(np.float32)
+        taps_h = rng.standard_normal((count, 2 * U + 2)).astype(np.float32)
+        blocks = torch.from_numpy(blocks_h).cuda()
+        taps = torch.from_numpy(taps_h).cuda()
         start = torch.from_numpy(rng.standard_normal((count, U)).astype(np.float32)).cuda()
         accumulate = call == 1
         ref = start.clone()
@@ -64,3 +89,5 @@ def test_noalloc_matches_fi_tau_on_two_calls_in_a_row(U, count):
         base = start.cpu().numpy() if accumulate else 0.0
         assert np.isfinite(g).all()
         assert rel(g - base, r - base) < TOL, (U, count, call)
+        rows, want = oracle_tau(blocks_h, taps_h, rng)
+        assert rel((g - base)[:, rows], want) < TOL, (U, count, call, "oracle")
