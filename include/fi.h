@@ -73,7 +73,12 @@ extern "C" {
 #define FI_PATH_WINDOW 0    /* default: one persistent kernel per aligned window of W
                                tokens (red cells + all blocks smaller than W, in shared
                                memory), one launch per larger block */
-#define FI_PATH_TOKEN 1     /* the pages' design: one launch sequence (graph) per token */
+#define FI_PATH_TOKEN 1     /* the pages' design ([Impl]): per token the step kernel (red
+                               cells of every layer), the block it releases over every
+                               layer, and an advance of the device-side step record; with
+                               graphs on, those launches are one captured CUDA graph per
+                               block size 2^q (one more for the last token), replayed per
+                               token with the token index read from device memory */
 #define FI_PATH_LAZY 2      /* baseline ([Base] "Lazy"): y^l_t summed over the whole history
                                when token t needs it, O(t) per token; one launch per token */
 #define FI_PATH_EAGER 3     /* baseline ([Base] "Eager"): each activation pushed onto every
@@ -175,7 +180,12 @@ int fi_set_stream(fi_ctx *ctx, void *stream);
    once; they take no graphs and record no trace. */
 int fi_set_path(fi_ctx *ctx, int path);
 
-/* Enable (1) or disable (0) replay of captured CUDA graphs ([Impl]). */
+/* Enable (1) or disable (0) replay of captured CUDA graphs ([Impl]).  Window path:
+ * the launch sequence of a whole call is captured once per call shape and replayed.
+ * Per-token path (and fi_step): one graph per block size, captured on first use and
+ * replayed per token.  With graphs off every launch is issued from the host.  Graphs
+ * are re-captured after fi_set_tau or fi_set_trace; the per-token graphs carry no trace
+ * events, so with tracing on the per-token path launches from the host. */
 int fi_set_graphs(fi_ctx *ctx, int on);
 
 /* Override the tau choice for block size 2^q (FI_TAU_AUTO restores the measured

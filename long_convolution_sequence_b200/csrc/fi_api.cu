@@ -119,6 +119,11 @@ struct fi_ctx {
     size_t pre_n = 0;
     std::map<GraphKey, GraphEntry> gcache;
     std::vector<GraphKey> gorder;
+    // per-token path: one graph per (mode, block size 2^q released after the token;
+    // index 32 = the last token, which releases none), replayed per token
+    TokIO* tio = nullptr;
+    cudaGraphExec_t tokg[2][33] = {};
+    long long tokg_nodes[2][33] = {};
     size_t bytes = 0;
     // tracing: per-launch event pairs grouped by kernel class
     int trace_on = 0;
@@ -522,9 +527,11 @@ TileArgs stack_tile_args(const fi_ctx* c, long long n) {
 
 // The gray blocks of every layer released after the n-th token, one launch
 // (section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)").
-int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st, int pdl = 0, int force_acc = 0) {
+int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st, int pdl = 0, int force_acc = 0,
+                 const TokIO* io = nullptr) {
     TileArgs a = stack_tile_args(c, n);
     if (force_acc) a.overwrite = 0;
+    a.io = io;  // replayed per-token graph: the kernels take n from the step record
     const int q = ctz64(n);
     const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
                     : (q <= fused_qmax() ? FI_K_BLOCK_FFT : FI_K_BLOCK_CLUSTER);
@@ -691,8 +698,10 @@ int tau_fft_noalloc_impl(int U, int q, int count, const float* blocks, const flo
 int tau_of(const fi_ctx* c, int q) { return c->tau_user[q] ? c->tau_user[q] : c->tau[q]; }
 
 // ---------------------------------------------------------------- launch sequences
-int enqueue_token(fi_ctx* c, long long t, const float* x, float* y, int closed, cudaStream_t st) {
+int enqueue_token(fi_ctx* c, long long t, const float* x, float* y, int closed, cudaStream_t st,
+                  const TokIO* io = nullptr) {
     StepArgs a;
+    a.io = io;
     a.act = c->act;
     a.h = c->h;
     a.M = c->M;
@@ -717,7 +726,73 @@ int enqueue_token(fi_ctx* c, long long t, const float* x, float* y, int closed, 
         k_token_step<kStepNT><<<grid, kStepNT, 0, st>>>(a);
         CK(cudaGetLastError());
     }
-    if (n < c->L && a.fuseU == 0) return launch_block(c, n, impl, st);
+    if (n < c->L && a.fuseU == 0) return launch_block(c, n, impl, st, 0, 0, io);
+    return FI_OK;
+}
+
+// The launches of one token step with the token taken from the step record: the step
+// kernel, the block released after it (edge 2^q; none for the last token), and the
+// advance of the record.  Captured once per (mode, q) into a graph.
+int capture_token_graph(fi_ctx* c, int closed, int idx) {
+    const long long t = idx == 32 ? c->L - 1 : (1LL << idx) - 1;  // a token releasing edge 2^idx
+    c->enq_launches = 0;
+    CK(cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed));
+    int rc = enqueue_token(c, t, nullptr, nullptr, closed, c->cap, c->tio);
+    if (!rc) {
+        k_advance_step<<<1, 1, 0, c->cap>>>(c->tio);
+        c->enq_launches++;
+    }
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(c->cap, &graph);
+    if (!rc && e == cudaSuccess) e = cudaGetLastError();
+    if (rc || e != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        cudaGetLastError();
+        return rc ? rc : set_err(FI_ECUDA, "token graph capture failed: %s", cudaGetErrorString(e));
+    }
+    const char* f = getenv("FI_FAULT");
+    if (f && strstr(f, "capture")) {
+        cudaGraphDestroy(graph);
+        return set_err(FI_ECUDA, "injected graph capture failure (FI_FAULT=capture)");
+    }
+    e = cudaGraphInstantiate(&c->tokg[closed][idx], graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) {
+        c->tokg[closed][idx] = nullptr;
+        return set_err(FI_ECUDA, "token graph instantiate failed: %s", cudaGetErrorString(e));
+    }
+    c->tokg_nodes[closed][idx] = c->enq_launches;
+    return FI_OK;
+}
+
+// The per-token path from captured graphs: the step record is set once for the call,
+// then one graph replay per token, the graph of the block size the token releases.
+int run_token_graphs(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed) {
+    for (long long t = t0; t < t0 + steps; ++t) {  // capture what this call needs first
+        const long long n = t + 1;
+        const int idx = n < c->L ? ctz64(n) : 32;
+        if (!c->tokg[closed][idx]) {
+            int rc = capture_token_graph(c, closed, idx);
+            if (rc) return rc;
+        }
+    }
+    TokIO v;
+    v.x = x;
+    v.y = out;
+    v.tx = t0;
+    v.t = t0;
+    v.closed = closed;
+    k_set_step<<<1, 1, 0, c->stream>>>(c->tio, v);
+    CK(cudaGetLastError());
+    long long nl = 1;
+    for (long long t = t0; t < t0 + steps; ++t) {
+        const long long n = t + 1;
+        const int idx = n < c->L ? ctz64(n) : 32;
+        CK(cudaGraphLaunch(c->tokg[closed][idx], c->stream));
+        nl += c->tokg_nodes[closed][idx];
+    }
+    c->launches += nl;
+    c->last_trace = nullptr;
     return FI_OK;
 }
 
@@ -774,6 +849,11 @@ void drop_graphs(fi_ctx* c) {
     for (auto& kv : c->gcache) cudaGraphExecDestroy(kv.second.exec);
     c->gcache.clear();
     c->gorder.clear();
+    for (int m = 0; m < 2; ++m)
+        for (int i = 0; i < 33; ++i) {
+            if (c->tokg[m][i]) cudaGraphExecDestroy(c->tokg[m][i]);
+            c->tokg[m][i] = nullptr;
+        }
 }
 
 // Run a launch sequence, from a captured graph when enabled (section
@@ -811,6 +891,7 @@ int run_baseline(fi_ctx* c, long long t0, long long steps, const float* x, float
 int run(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed) {
     if (c->path >= FI_PATH_LAZY) return run_baseline(c, t0, steps, x, out, closed);
     const bool window = c->path == FI_PATH_WINDOW && c->W > 0;
+    if (!window && c->graphs && !c->trace_on) return run_token_graphs(c, t0, steps, x, out, closed);
     c->enq_launches = 0;
     if (!c->graphs || !window) {
         c->eager_trace.clear();
@@ -982,6 +1063,7 @@ void free_ctx(fi_ctx* c) {
     cudaFree(c->sx);
     cudaFree(c->sy);
     cudaFree(c->pre);
+    cudaFree(c->tio);
     for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
     if (c->cap) cudaStreamDestroy(c->cap);
     c->magic = 0;
@@ -999,6 +1081,7 @@ int create_impl(fi_ctx* c, const float* filters) {
     int rc;
     if ((rc = dev_alloc(c, &c->act, (size_t)(M + 1) * G * L))) return rc;
     if ((rc = dev_alloc(c, &c->h, (size_t)M * D * L))) return rc;
+    if ((rc = dev_alloc(c, &c->tio, 1))) return rc;
     CK(cudaMemcpyAsync(c->h, filters, sizeof(float) * M * D * L, cudaMemcpyDefault, c->cap));
     // twiddles from fp64 host trigonometry
     if ((rc = upload_twiddles(c))) return rc;

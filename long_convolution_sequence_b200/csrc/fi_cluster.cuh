@@ -109,7 +109,8 @@ __device__ __forceinline__ void cluster_partner(int k1, int k2, int* pk1, int* p
 
 template <int LOGNC, int LOGN2, int TWLOG>
 __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGNC, LOGN2>::MINB)
-    k_block_fft_cluster(TileArgs a) {
+    k_block_fft_cluster(TileArgs a0) {
+    const TileArgs a = with_step(a0);
     namespace cg = cooperative_groups;
     using G = ClusterTile<LOGNC, LOGN2>;
     constexpr int NC = G::NC, N2 = G::N2, N = G::N, LOGN = G::LOGN, T = G::T, R0 = G::R0, NP = G::NP;

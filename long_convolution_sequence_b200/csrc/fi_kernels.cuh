@@ -85,6 +85,23 @@ __device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(
 __device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
 __device__ __forceinline__ float2 conjf2(float2 a) { return make_float2(a.x, -a.y); }
 
+// ----------------------------------------------------------------- per-token step state
+// The per-token path replays one captured CUDA graph per block size (section
+// "Implementierungsdetails": the launches of one token step are recorded once and
+// replayed), so the token a replay works on cannot be a kernel argument: it lives in
+// this device-side record, written by k_set_step at the start of a call and advanced
+// by k_advance_step at the end of every token.
+struct TokIO {
+    const float* x;  // teacher: tokens [.][G] from token tx on; closed loop: [G] token tx, or null
+    float* y;        // y^M [.][G] from token tx on
+    long long tx;    // token of x[0] / y[0]
+    long long t;     // token being processed
+    int closed;
+};
+
+__global__ void k_set_step(TokIO* io, TokIO v) { *io = v; }
+__global__ void k_advance_step(TokIO* io) { io->t += 1; }
+
 // ----------------------------------------------------------------- tile addressing
 // A "tile" is one gray block for one (layer, chain), or one stand-alone tau item.
 struct TileArgs {
@@ -109,7 +126,17 @@ struct TileArgs {
     long long spec_stride;  // complex entries per item
     const float2* tw;    // e^{-2 pi i k / 2^twlog}, k < 2^twlog
     int twlog;
+    const TokIO* io;     // non-null: n = io->t + 1 (replayed per-token graph), overwrite = n a power of 2
 };
+
+// The block position of a launch: from the arguments, or from the step record.
+__device__ __forceinline__ TileArgs with_step(TileArgs a) {
+    if (a.io) {
+        a.n = a.io->t + 1;
+        a.overwrite = (a.n & (a.n - 1)) == 0;
+    }
+    return a;
+}
 
 struct TilePtrs {
     const float* in;
@@ -141,7 +168,8 @@ __device__ __forceinline__ TilePtrs tile_ptrs(const TileArgs& a, long long item)
 // out[r] (+)= sum_{j<U} in[j] * taps[U + r - j], one tile per CTA, operands staged
 // in shared memory (block U floats, taps 2U floats).
 template <int NT, int RG>
-__global__ void __launch_bounds__(NT) k_tile_direct(TileArgs a) {
+__global__ void __launch_bounds__(NT) k_tile_direct(TileArgs a0) {
+    const TileArgs a = with_step(a0);
     extern __shared__ float sm[];
     const int U = a.U;
     float* sin = sm;
@@ -344,7 +372,8 @@ __device__ __forceinline__ void fft_last_pass_store(const float2* X, int t, int 
 }
 
 template <int LOGN, int TWLOG>
-__global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_block_fft(TileArgs a) {
+__global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_block_fft(TileArgs a0) {
+    const TileArgs a = with_step(a0);
     using G = FftTile<LOGN>;
     constexpr int N = G::N, RB = G::RB, R0 = G::R0, T = G::T, NP = G::NP, LOGRB = G::LOGRB;
     extern __shared__ __align__(16) float2 fft_sm[];
@@ -506,18 +535,27 @@ struct StepArgs {
     float* y;        // [G] y^M_t
     int closed;      // write a^M_t as token t+1
     int fuseU;       // edge of the block n = t+1 done here (0: none)
+    const TokIO* io; // non-null: t, x and y come from the step record (replayed graph)
 };
 
 template <int NT>
 __global__ void __launch_bounds__(NT) k_token_step(StepArgs a) {
     const long long g0 = (long long)blockIdx.x * 32;
     const int lane = threadIdx.x;
-    const long long t = a.t;
+    long long t = a.t;
+    const float* xt = a.x;
+    float* yt = a.y;
+    if (a.io) {
+        const TokIO io = *a.io;
+        t = io.t;
+        yt = io.y + (t - io.tx) * a.G;
+        xt = io.closed ? (t == io.tx ? io.x : nullptr) : io.x + (t - io.tx) * a.G;
+    }
     if (lane < 32) {
         const long long g = g0 + lane;
         if (g < a.G) {
             const long long c = g % a.D;
-            float av = a.x ? a.x[g] : a.act[g * a.L + t];
+            float av = xt ? xt[g] : a.act[g * a.L + t];
             a.act[g * a.L + t] = av;
             float y = 0.f;
             for (int l = 1; l <= a.M; ++l) {
@@ -528,7 +566,7 @@ __global__ void __launch_bounds__(NT) k_token_step(StepArgs a) {
                 av = act_tanh(y);
                 *slot = av;
             }
-            a.y[g] = y;
+            yt[g] = y;
             if (a.closed && t + 1 < a.L) a.act[g * a.L + t + 1] = av;
         }
     }

@@ -247,6 +247,66 @@ def test_generate_continues_across_calls_and_reset_repeats(window):
     assert rel(runs[0], ref) < TOL_CL
 
 
+@pytest.mark.parametrize("closed", [True, False])
+def test_token_path_graphs_replay_the_eager_launches(closed):
+    # the per-token path from one captured graph per block size must compute exactly
+    # what the same launches issued from the host compute, and match the oracle
+    M, B, D, L = 3, 2, 5, 2048
+    h = synth.filters(M, D, L, seed=8)
+    x0 = synth.start_token(B, D, seed=8)
+    x = synth.inputs(L, B, D, seed=8)
+    if closed:
+        ref = oracle.stack(h, x0, T=L, closed_loop=True, want=("y_last",))["y_last"]
+    else:
+        ref = oracle.stack(h, x, want=("y_last",))["y_last"]
+    outs = []
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        ctx.set_path(fi.FI_PATH_TOKEN)
+        for graphs in (True, False, True):
+            ctx.reset()
+            ctx.set_graphs(graphs)
+            n0 = ctx.info().launches
+            y = np.empty((L, B, D), np.float32)
+            if closed:
+                ctx.generate(x0, 700, y[:700])           # two calls: the step record is
+                ctx.generate(None, L - 700, y[700:])      # set again by the second
+            else:
+                ctx.forward(x[:700], 700, y[:700])
+                ctx.forward(x[700:], L - 700, y[700:])
+            if graphs:
+                # per token: step kernel, block launch unless fused into it, advance;
+                # per call one record write
+                assert L * 2 + 2 <= ctx.info().launches - n0 <= L * 3 + 2
+            outs.append(y)
+    np.testing.assert_array_equal(outs[0], outs[1])
+    np.testing.assert_array_equal(outs[0], outs[2])
+    assert rel(outs[0], ref) < (TOL_CL if closed else TOL_TF)
+
+
+def test_step_calls_with_changing_pointers_replay_graphs():
+    # fi_step: every call names new input and output buffers (device and host); the
+    # replayed graphs read them from the step record
+    M, B, D, L = 2, 1, 6, 512
+    h = synth.filters(M, D, L, seed=9)
+    x = synth.inputs(L, B, D, seed=9)
+    ref = oracle.stack(h, x, want=("y_last",))["y_last"]
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        xd = dev(x)
+        yd = torch.empty((L, B, D), device="cuda")
+        yh = np.empty((L, B, D), np.float32)
+        for t in range(L):
+            if t % 3 == 0:
+                ctx.step(np.ascontiguousarray(x[t]), yh[t])
+            else:
+                ctx.step(xd[t], yd[t])
+        torch.cuda.synchronize()
+        got = yd.cpu().numpy()
+        for t in range(0, L, 3):
+            got[t] = yh[t]
+        assert ctx.info().t == L
+    assert rel(got, ref) < TOL_TF
+
+
 @pytest.mark.parametrize("force", ["direct", "fft"])
 def test_forced_tau_everywhere(force, window):
     window(32)
