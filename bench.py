@@ -222,9 +222,18 @@ def main():
     ap.add_argument("--sweep-b", default="1,2,4,8")
     ap.add_argument("--sweep-d", default="256,512,768,1024")
     ap.add_argument("--sweep-l", default="12,14,16,18", help="log2 L values")
-    ap.add_argument("--baseline", choices=("lazy", "eager"),
+    ap.add_argument("--baseline", choices=("lazy", "eager", "lazy_np", "eager_np"),
                     help="time the pages' Lazy or Eager baseline on this device next to the tiled path "
                          "(default workload: short)")
+    ap.add_argument("--ablation", choices=("layers", "graphs", "tau", "latency"),
+                    help="the pages' ablations on this path: one across-layer block launch against M "
+                         "per-layer launches, graphs on against off, Hybrid tau against FFT-only and "
+                         "direct-only, the per-token latency distribution; one JSON line per variant")
+    ap.add_argument("--baseline-workload", default="short", choices=sorted(WORKLOADS),
+                    help="workload of --baseline (the O(L^2) baselines take minutes at the headline length)")
+    ap.add_argument("--lm", action="store_true",
+                    help="the Hyena-like language model end to end (18 layers, B=4, D=768, L=2^15, vocabulary "
+                         "50257, greedy decoding): tokens/s and the mixer / non-mixer split")
     ap.add_argument("--prefill", default=None,
                     help="comma-separated prompt lengths: time fi_prefill against the online "
                          "teacher-forced path over the same prompt (headline stack)")
@@ -235,6 +244,10 @@ def main():
         return bench_sweep(args)
     if args.baseline:
         return bench_baseline(args)
+    if args.ablation:
+        return bench_ablation(args)
+    if args.lm:
+        return bench_lm(args)
     M, B, D, L = WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -502,16 +515,17 @@ def bench_sweep(args):
 
 
 def bench_baseline(args):
-    """The pages' parallel Lazy or Eager baseline (FI_PATH_LAZY / FI_PATH_EAGER) timed
-    on this device beside the tiled window path, same workload, same process: one
-    closed-loop generation each after warm-up, CUDA events.  Both baselines cost O(L^2)
-    per channel-layer, so the headline length (2^17) is out of reach in minutes; the
-    default workload is the headline stack at L = 2^14, and the line also carries the
-    baseline's time scaled to L = 2^17 by the L^2 law (labelled as extrapolated)."""
+    """One of the pages' Lazy or Eager baselines (FI_PATH_LAZY / FI_PATH_EAGER, parallel
+    across layers, or their NP forms FI_PATH_LAZY_NP / FI_PATH_EAGER_NP) timed on this
+    device beside the tiled window path, same workload, same process: one closed-loop
+    generation each after warm-up, CUDA events.  The baselines cost O(L^2) per
+    channel-layer; the default workload (--baseline-workload) is the headline stack at
+    L = 2^14, where the line also carries the baseline's time scaled to L = 2^17 by the
+    L^2 law (labelled as extrapolated); --baseline-workload headline measures it."""
     import torch
     import long_convolution_sequence_b200 as fi
     from long_convolution_sequence_b200 import synth
-    wl = args.workload if args.workload != "headline" else "short"
+    wl = args.baseline_workload
     M, B, D, L = WORKLOADS[wl]
     h = synth.filters(M, D, L, seed=0)
     x0 = torch.from_numpy(synth.start_token(B, D, seed=0)).cuda()
@@ -531,7 +545,8 @@ def bench_baseline(args):
     timed(3)
     fi_ms = timed(3)
     ctx.reset()
-    ctx.set_path(fi.FI_PATH_LAZY if args.baseline == "lazy" else fi.FI_PATH_EAGER)
+    ctx.set_path({"lazy": fi.FI_PATH_LAZY, "eager": fi.FI_PATH_EAGER, "lazy_np": fi.FI_PATH_LAZY_NP,
+                  "eager_np": fi.FI_PATH_EAGER_NP}[args.baseline])
     ctx.generate(x0, min(L, 256), out)  # warm-up of the baseline's kernels
     torch.cuda.synchronize()
     base_ms = timed(1)
@@ -549,6 +564,201 @@ def bench_baseline(args):
     print(json.dumps(line), flush=True)
     return 0
 
+
+
+def bench_ablation(args):
+    """The pages' ablations ("Ablationsstudien", "Implementierungsdetails", "Antwortzeit
+    pro Token") measured on this path, on the workload's stack (default: headline),
+    closed loop from t = 0, CUDA events, one warm-up and two timed generations per
+    variant; one JSON line per variant.
+
+    layers:  every block launch covering all M layers (Algorithm 3) against M launches
+             of one layer each (FI_LAYER_SPLIT=1), on the window and per-token paths;
+    graphs:  captured CUDA graphs against launches issued from the host, both paths;
+    tau:     the measured Hybrid choice against FFT for every size it serves (U >= 8)
+             and direct for every size it serves (U <= 4096), both paths (on the window
+             path every block smaller than W runs inside the window kernel, so tau only
+             chooses among the larger sizes there);
+    latency: device time per token from a traced generation: per-token path, each
+             token's launches; window path, each window launch spread over its W tokens
+             plus the block launch at the window's end on its last token."""
+    import torch
+    import long_convolution_sequence_b200 as fi
+    from long_convolution_sequence_b200 import synth
+    M, B, D, L = WORKLOADS[args.workload]
+    h = synth.filters(M, D, L, seed=0)
+    x0 = torch.from_numpy(synth.start_token(B, D, seed=0)).cuda()
+    out = torch.empty((L, B, D), device="cuda")
+    paths = {"window": fi.FI_PATH_WINDOW, "token": fi.FI_PATH_TOKEN}
+
+    def timed(ctx, n=2):
+        ctx.reset()
+        ctx.generate(x0, L, out)
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for _ in range(n):
+            ctx.reset()
+            ctx.generate(x0, L, out)
+        ev1.record()
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1) / n
+
+    def emit(variant, path, ms, **extra):
+        line = {"metric": "ablation: mixer tokens/s", "ablation": args.ablation, "variant": variant,
+                "path": path, "ms_per_generation": round(ms, 3), "value": round(B * L / (ms / 1e3), 1),
+                "unit": "tokens/s", "finite": bool(torch.isfinite(out).all().item()),
+                "config": {"workload": args.workload, "layers": M, "B": B, "D": D, "L": L}}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+
+    if args.ablation == "layers":
+        for split in (0, 1):
+            os.environ["FI_LAYER_SPLIT"] = str(split)
+            with fi.FlashInference(M, B, D, L, h) as ctx:
+                for pname, path in paths.items():
+                    ctx.set_path(path)
+                    n0 = ctx.info().launches
+                    ms = timed(ctx)
+                    emit("per-layer block launches" if split else "one launch for all layers", pname, ms,
+                         launches_per_generation=(ctx.info().launches - n0) // 3)
+        os.environ.pop("FI_LAYER_SPLIT", None)
+        return 0
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        info = ctx.info()
+        P = L.bit_length() - 1
+        if args.ablation == "graphs":
+            for pname, path in paths.items():
+                ctx.set_path(path)
+                for graphs in (True, False):
+                    ctx.set_graphs(graphs)
+                    n0 = ctx.info().launches
+                    ms = timed(ctx, 1)
+                    emit("graphs on" if graphs else "graphs off", pname, ms,
+                         launches_per_generation=(ctx.info().launches - n0) // 2)
+            return 0
+        if args.ablation == "tau":
+            choices = {"hybrid (measured)": {},
+                       "fft everywhere": {q: fi.FI_TAU_FFT for q in range(3, P)},
+                       "direct everywhere": {q: fi.FI_TAU_DIRECT for q in range(0, min(P, 13))}}
+            for pname, path in paths.items():
+                ctx.set_path(path)
+                for name, table in choices.items():
+                    for q in range(P):
+                        ctx.set_tau(q, fi.FI_TAU_AUTO)
+                    for q, impl in table.items():
+                        ctx.set_tau(q, impl)
+                    tau = {str(q): ("fft" if ctx.info().tau[q] == fi.FI_TAU_FFT else "direct") for q in range(P)}
+                    emit(name, pname, timed(ctx), tau=tau)
+            for q in range(P):
+                ctx.set_tau(q, fi.FI_TAU_AUTO)
+            return 0
+        # latency
+        for pname, path in paths.items():
+            ctx.set_path(path)
+            ctx.set_trace(True)
+            ctx.reset()
+            ctx.generate(x0, L, out)
+            torch.cuda.synchronize()
+            cls, qs, us = ctx.trace_launches()
+            per_tok = np.zeros(L)
+            W = info.window
+            if path == fi.FI_PATH_WINDOW:
+                t = 0
+                for c, q, u in zip(cls, qs, us):
+                    if c == fi.FI_K_WINDOW:
+                        per_tok[t:t + W] += u / W
+                        t += W
+                    else:  # the block released at the end of the window just done
+                        per_tok[t - 1] += u
+            else:
+                t = -1
+                for c, q, u in zip(cls, qs, us):
+                    if c == fi.FI_K_TOKEN_STEP:
+                        t += 1
+                    per_tok[t] += u
+            ctx.set_trace(False)
+            n = np.arange(1, L + 1)
+            lowq = np.array([(int(v) & -int(v)).bit_length() - 1 for v in n])
+            by_q = {str(q): round(float(per_tok[lowq == q].mean()), 3) for q in range(P + 1) if (lowq == q).any()}
+            pct = {p: round(float(np.percentile(per_tok, p)), 3) for p in (50, 90, 99, 99.9)}
+            emit("per-token device time", pname, float(per_tok.sum()) / 1e3,
+                 us_per_token={"mean": round(float(per_tok.mean()), 3), "percentiles": pct,
+                               "max": round(float(per_tok.max()), 1),
+                               "mean_by_released_block_log2": by_q},
+                 note="time of one traced generation (events around every launch)")
+        return 0
+
+
+LM_CONFIG = dict(M=18, B=4, D=768, L=1 << 15, V=50257)
+
+
+def bench_lm(args):
+    """The Hyena-like model end to end (BASELINE configuration 5): greedy generation of
+    L tokens from uniform random start tokens, random-init weights (bf16 GEMMs, fp32
+    mixer).  One warm-up generation, then timed generations (CUDA events); a traced
+    generation gives the mixers' share of the device time (the pages' mixer / non-mixer
+    split, section "Hauptergebnisse"); the oracle is timed on its first tokens."""
+    import torch
+    import long_convolution_sequence_b200 as fi
+    from long_convolution_sequence_b200 import synth
+    c = LM_CONFIG
+    M, B, D, L, V = c["M"], c["B"], c["D"], c["L"], c["V"]
+    t0 = time.perf_counter()
+    p = synth.hyena_params(M, D, L, V, seed=0)
+    t_gen = time.perf_counter() - t0
+    tok0 = synth.token_ids(1, B, V, seed=0)[0]
+    stack = lambda k: np.ascontiguousarray(np.stack(p[k]))
+    lm = fi.LanguageModel(M, B, D, L, V, p["E"], p["W_lm"], stack("W_in"), stack("c"), stack("W1"), stack("W2"),
+                          stack("h"))
+    tok0_d = torch.from_numpy(tok0).cuda()
+    nxt = torch.empty((L, B), dtype=torch.int32, device="cuda")
+
+    def gen():
+        lm.reset()
+        lm.generate(tok0_d, L, nxt)
+
+    gen()
+    torch.cuda.synchronize()
+    clocks = Clocks(0)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(args.steps, 2))
+    ev0.record()
+    for _ in range(steps):
+        gen()
+    ev1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / steps
+    lm.set_trace(True)
+    gen()
+    torch.cuda.synchronize()
+    mix_us, tot_us = lm.split()
+    lm.set_trace(False)
+    toks = nxt.cpu().numpy()
+    lm.close()
+    # the oracle on a bounded sample: the first T_s tokens of the same generation
+    from oracle import hyena
+    T_s = 8
+    t1 = time.perf_counter()
+    ref = hyena.run(p, tok0=tok0, T=T_s, want=("tokens",))
+    sec = time.perf_counter() - t1
+    line = {"metric": "end-to-end tokens/s (B*L/time), Hyena-like model, greedy decoding", "value": round(B * L / (ms / 1e3), 1),
+            "unit": "tokens/s", "ms_per_generation": round(ms, 1), "steps": steps, "dtype": "bf16 GEMMs / f32 mixer",
+            "data": "synthetic: random-init weights, uniform random start tokens",
+            "config": {"workload": "Hyena-like model, %d layers, B=%d, D=%d, L=%d, vocabulary %d" % (M, B, D, L, V),
+                       **c},
+            "mixer_share": {"mixer_us": round(mix_us, 1), "total_us": round(tot_us, 1),
+                            "frac": round(mix_us / tot_us, 4) if tot_us else None,
+                            "note": "traced generation: events around every block launch and the mixer steps of "
+                                    "every 64th token (scaled)"},
+            "greedy_matches_oracle_first_tokens": bool((toks[:T_s] == ref["next"]).all()),
+            "cpu_baseline": {"value": round(B * T_s / sec, 3), "unit": "tokens/s", "kind": "oracle",
+                             "cores": 1, "sample": "first %d tokens of the same generation (fp64 numpy)" % T_s},
+            "clocks": clk, "setup_s": {"params": round(t_gen, 1)}}
+    print(json.dumps(line), flush=True)
+    return 0
 
 def bench_prefill(args):
     """Prompt prefill (fi_prefill: one FFT convolution per layer) against the online

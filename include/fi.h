@@ -83,6 +83,10 @@ extern "C" {
                                when token t needs it, O(t) per token; one launch per token */
 #define FI_PATH_EAGER 3     /* baseline ([Base] "Eager"): each activation pushed onto every
                                later position as soon as it is known, O(L-t) per token */
+#define FI_PATH_LAZY_NP 4   /* baseline ([Base] "Lazy NP"): Lazy without cross-layer
+                               parallelism, one launch per layer and token, in layer order */
+#define FI_PATH_EAGER_NP 5  /* baseline ([Base] "Eager NP"): Eager without cross-layer
+                               parallelism, one launch per layer and token, in layer order */
 
 typedef struct fi_ctx fi_ctx;
 
@@ -173,11 +177,13 @@ int fi_read_layer(fi_ctx *ctx, int layer, int t0, int t1, float *dst);
 int fi_set_stream(fi_ctx *ctx, void *stream);
 
 /* Choose the execution path (FI_PATH_*).  The two tiled paths (WINDOW, TOKEN) share
-   their buffer state and may be switched at any token; LAZY and EAGER keep their own
-   state, so a change to or from them is accepted only at t = 0 (after fi_create or
-   fi_reset), else FI_EINVAL.  LAZY and EAGER are the pages' parallel baselines: the
-   part of token t that does not depend on its own layer chain runs for every layer at
-   once; they take no graphs and record no trace. */
+   their buffer state and may be switched at any token; the baselines (LAZY, EAGER and
+   their NP forms) keep their own state, so a change to or from them is accepted only
+   at t = 0 (after fi_create or fi_reset), else FI_EINVAL.  LAZY and EAGER are the
+   pages' parallel baselines: the part of token t that does not depend on its own layer
+   chain runs for every layer at once; LAZY_NP and EAGER_NP do each layer's share as a
+   launch of its own, layer after layer.  The baselines take no graphs and record no
+   trace. */
 int fi_set_path(fi_ctx *ctx, int path);
 
 /* Enable (1) or disable (0) replay of captured CUDA graphs ([Impl]).  Window path:
@@ -200,6 +206,13 @@ int fi_set_trace(fi_ctx *ctx, int on);
 /* Per kernel class: launches and device time of the most recent run (fi_step,
  * fi_generate or fi_forward call) made with tracing on.  Synchronises the stream. */
 int fi_trace_read(fi_ctx *ctx, fi_trace *out);
+
+/* The launches of the most recent traced run, in issue order: kernel class (FI_K_*),
+ * block size exponent q (-1 for launches that are not block launches) and device time
+ * in microseconds of launch i in cls[i], q[i], us[i] for i < max.  Returns the number of
+ * launches the run made (which may exceed max), or a negative FI_E* code.  Synchronises
+ * the stream. */
+int fi_trace_launches(fi_ctx *ctx, int max, int *cls, int *q, float *us);
 
 /* Fill *info with the context's shape, state and tau table. */
 int fi_get_info(const fi_ctx *ctx, fi_info *info);
@@ -242,6 +255,53 @@ int fi_tau(int impl, int U, int count, const float *blocks, const float *taps, i
  * completion.  FI_EINVAL for U beyond 65536 (or any fi_tau argument error). */
 int fi_tau_fft_noalloc(int U, int count, const float *blocks, const float *taps, int ldt,
                        float *out, int accumulate);
+
+/* ---------------------------------------------------------------- language model
+ * A Hyena-like language model built around the mixer: the pages describe an LCSM layer
+ * as the mixer followed by a block with "MLP, Schicht-Normalisierung, etc." (section
+ * "Modellarchitektur") and measure a Hyena model with random weights end to end
+ * (sections "Experimentelle Einrichtung", "Hauptergebnisse").  Per token t, batch row b
+ * (u: residual stream of D values; LN: layer norm without affine parameters, eps 1e-5;
+ * bf16(.): rounding to bfloat16, the operand of a bf16 GEMM with fp32 accumulation):
+ *   u = E[tok_t];  for each layer l:
+ *     z = W_in^l bf16(LN(u)) = (q, k, v);   zc_t = c0 z_t + c1 z_{t-1} + c2 z_{t-2}
+ *     x_t = kc vc;   y_t = sum_{s<=t} h^l[t-s] x_s  (the mixer, fp32, relaxed tiling)
+ *     u += qc y_t;   u += W2^l bf16(GELU(W1^l bf16(LN(u))))
+ *   logits = W_lm bf16(LN(u));   greedy: tok_{t+1} = argmax (lowest id among equal maxima)
+ * Weights arrive as fp32 arrays holding bf16 values (host or device), row-major:
+ * E, W_lm [V][D]; W_in [layers][3D][D]; conv [layers][3][3D] (taps c0, c1, c2, fp32);
+ * W1 [layers][4D][D]; W2 [layers][D][4D]; filters [layers][D][L] fp32.  They are copied.
+ * 1 <= B <= 8, D a multiple of 8, L a power of two.  Token arrays are int32, host or
+ * device.  Returns NULL on error (fi_last_error). */
+typedef struct fi_lm fi_lm;
+fi_lm *fi_lm_create(int layers, int B, int D, int L, int V, const float *E, const float *W_lm,
+                    const float *W_in, const float *conv, const float *W1, const float *W2,
+                    const float *filters);
+
+/* Release the model.  NULL is accepted. */
+void fi_lm_destroy(fi_lm *m);
+
+/* Rewind to t = 0 (a new sequence; the short-convolution history restarts at zero). */
+int fi_lm_reset(fi_lm *m);
+
+/* Teacher-forced tokens t .. t+steps-1: tokens [steps][B] are the inputs; logits
+ * [steps][B][V] receives the logits (NULL: not returned); next [steps][B] the greedy
+ * choices.  FI_ECAPACITY past L. */
+int fi_lm_forward(fi_lm *m, const int *tokens, int steps, float *logits, int *next);
+
+/* Greedy generation of `steps` tokens: tok0 [B] is the input at the current position
+ * (NULL: continue from the previous call's last choice; required at t = 0); next
+ * [steps][B] receives each step's choice, which is the following step's input. */
+int fi_lm_generate(fi_lm *m, const int *tok0, int steps, int *next);
+
+/* Tracing (off by default): later calls record events around every block launch of
+ * the mixers and around the mixer steps of every 64th token. */
+int fi_lm_set_trace(fi_lm *m, int on);
+
+/* Of the most recent traced call: its device time (total_us) and the part spent in
+ * the mixers (mixer_us: the block launches, plus the sampled mixer steps scaled to
+ * every token).  Synchronises. */
+int fi_lm_split(fi_lm *m, double *mixer_us, double *total_us);
 
 /* Message of the last failure on the calling thread ("" if none). */
 const char *fi_last_error(void);

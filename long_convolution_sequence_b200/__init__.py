@@ -14,7 +14,7 @@ _LIB_PATH = Path(__file__).resolve().parent / "libfi.so"
 
 FI_OK, FI_EINVAL, FI_ECAPACITY, FI_ENOMEM, FI_ECUDA, FI_ESTATE = 0, -1, -2, -3, -4, -5
 FI_TAU_AUTO, FI_TAU_DIRECT, FI_TAU_FFT = 0, 1, 2
-FI_PATH_WINDOW, FI_PATH_TOKEN, FI_PATH_LAZY, FI_PATH_EAGER = 0, 1, 2, 3
+FI_PATH_WINDOW, FI_PATH_TOKEN, FI_PATH_LAZY, FI_PATH_EAGER, FI_PATH_LAZY_NP, FI_PATH_EAGER_NP = range(6)
 
 
 class FiError(RuntimeError):
@@ -62,8 +62,16 @@ SIGNATURES = {
     "fi_set_trace": (_I, [_P, _I]),
     "fi_trace_read": (_I, [_P, ctypes.POINTER(fi_trace)]),
     "fi_debug_schedule": (_I, [_P, _I] + [ctypes.POINTER(_I)] * 5),
+    "fi_trace_launches": (_I, [_P, _I, _P, _P, _P]),
     "fi_tau": (_I, [_I, _I, _I, _P, _P, _I, _P, _I]),
     "fi_tau_fft_noalloc": (_I, [_I, _I, _P, _P, _I, _P, _I]),
+    "fi_lm_create": (_P, [_I, _I, _I, _I, _I] + [_P] * 7),
+    "fi_lm_destroy": (None, [_P]),
+    "fi_lm_reset": (_I, [_P]),
+    "fi_lm_forward": (_I, [_P, _P, _I, _P, _P]),
+    "fi_lm_generate": (_I, [_P, _P, _I, _P]),
+    "fi_lm_set_trace": (_I, [_P, _I]),
+    "fi_lm_split": (_I, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     "fi_last_error": (ctypes.c_char_p, []),
     "fi_version": (ctypes.c_char_p, []),
 }
@@ -190,6 +198,21 @@ class FlashInference:
             return cls
         return cls, {q: (tr.block_launches[q], tr.block_us[q]) for q in range(32) if tr.block_launches[q]}
 
+    def trace_launches(self):
+        """(cls, q, us) numpy arrays of every launch of the last traced run, in issue order."""
+        import numpy as np
+        lib = get_lib()
+        n = lib.fi_trace_launches(self._h, 0, None, None, None)
+        if n < 0:
+            _check(n)
+        cls = np.empty(max(n, 1), np.int32)
+        q = np.empty(max(n, 1), np.int32)
+        us = np.empty(max(n, 1), np.float32)
+        got = lib.fi_trace_launches(self._h, n, cls.ctypes.data, q.ctypes.data, us.ctypes.data)
+        if got < 0:
+            _check(got)
+        return cls[:n], q[:n], us[:n]
+
     def info(self) -> fi_info:
         inf = fi_info()
         _check(get_lib().fi_get_info(self._h, ctypes.byref(inf)))
@@ -200,6 +223,63 @@ class FlashInference:
         _check(get_lib().fi_debug_schedule(self._h, n, *[ctypes.byref(v) for v in vals]))
         U, impl, src_lo, dst_lo, dst_hi = (v.value for v in vals)
         return dict(U=U, impl=impl, src_lo=src_lo, dst_lo=dst_lo, dst_hi=dst_hi)
+
+
+def _iptr(a):
+    """Address of a contiguous int32 torch tensor / numpy array (None -> NULL)."""
+    if a is None:
+        return None
+    if hasattr(a, "data_ptr"):
+        assert a.is_contiguous() and str(a.dtype) == "torch.int32", "int32 contiguous tensor expected"
+        return a.data_ptr()
+    import numpy as np
+    assert isinstance(a, np.ndarray) and a.dtype == np.int32 and a.flags.c_contiguous
+    return a.ctypes.data
+
+
+class LanguageModel:
+    """The Hyena-like model around the mixer (fi_lm_create .. fi_lm_destroy); weights as
+    float32 arrays (bf16 values for the GEMM weights), per layer stacked: see fi.h."""
+
+    def __init__(self, layers, B, D, L, V, E, W_lm, W_in, conv, W1, W2, filters):
+        self.layers, self.B, self.D, self.L, self.V = layers, B, D, L, V
+        lib = get_lib()
+        h = lib.fi_lm_create(layers, B, D, L, V, *(_ptr(a) for a in (E, W_lm, W_in, conv, W1, W2, filters)))
+        if not h:
+            raise FiError(FI_EINVAL, last_error())
+        self._h = h
+        self._lib = lib
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.fi_lm_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def reset(self):
+        _check(get_lib().fi_lm_reset(self._h))
+
+    def forward(self, tokens, steps, logits, next_tokens):
+        _check(get_lib().fi_lm_forward(self._h, _iptr(tokens), steps, _ptr(logits), _iptr(next_tokens)))
+
+    def generate(self, tok0, steps, next_tokens):
+        _check(get_lib().fi_lm_generate(self._h, _iptr(tok0), steps, _iptr(next_tokens)))
+
+    def set_trace(self, on: bool):
+        _check(get_lib().fi_lm_set_trace(self._h, int(bool(on))))
+
+    def split(self):
+        """(mixer_us, total_us) of the last traced call."""
+        a, b = ctypes.c_double(), ctypes.c_double()
+        _check(get_lib().fi_lm_split(self._h, ctypes.byref(a), ctypes.byref(b)))
+        return a.value, b.value
 
 
 def tau(impl: int, U: int, blocks, taps, out, accumulate: bool = False):

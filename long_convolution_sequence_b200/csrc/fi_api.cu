@@ -26,6 +26,7 @@
 
 #include "fi.h"
 #include "fi_kernels.cuh"
+#include "fi_lm.cuh"
 
 using namespace fi;
 
@@ -100,6 +101,7 @@ struct fi_ctx {
     cudaStream_t stream = nullptr;   // user stream (nullptr = legacy default)
     cudaStream_t cap = nullptr;      // private stream used to capture graphs
     float* act = nullptr;            // [(M+1)][G][L]
+    float* yout = nullptr;           // language model: the mixers' outputs [M][G][L] (blocks read act[l], add onto yout[l])
     float* h = nullptr;              // [M][D][L]
     float2* tw = nullptr;            // [2^kTwLog]
     float2* spec[32] = {};           // per block size 2^q
@@ -110,6 +112,7 @@ struct fi_ctx {
     size_t win_smem = 0;
     int path = FI_PATH_WINDOW, graphs = 1;
     int pdl = 1;  // window-path launches overlap their start with the predecessor's end
+    int layer_split = 0;  // ablation (FI_LAYER_SPLIT=1): one block launch per layer instead of one for all
     long long t = 0;
     float* sx = nullptr;  // staging for host inputs
     size_t sx_n = 0;
@@ -170,10 +173,22 @@ int check_ctx(const fi_ctx* c) {
 cudaEvent_t pool_event(fi_ctx* c) {
     if (c->event_next == c->event_pool.size()) {
         cudaEvent_t e;
-        if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            cudaGetLastError();  // out of events: the launch goes untraced, no error is left behind
+            return nullptr;
+        }
         c->event_pool.push_back(e);
     }
     return c->event_pool[c->event_next++];
+}
+
+// Record an event on st: as an external event node while st is being captured into a
+// graph (so that the event is recorded at every replay), as a plain record otherwise.
+void trace_record(cudaEvent_t e, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) cudaGetLastError();
+    if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    else cudaEventRecord(e, st);
 }
 
 // Bracket one launch with events when tracing (also inside graph capture).
@@ -191,13 +206,12 @@ struct LaunchScope {
             r.a = pool_event(c);
             r.b = pool_event(c);
             on = r.a && r.b;
-            // external records become event nodes when the stream is being captured
-            if (on) cudaEventRecordWithFlags(r.a, st, cudaEventRecordExternal);
+            if (on) trace_record(r.a, st);
         }
     }
     ~LaunchScope() {
         if (on) {
-            cudaEventRecordWithFlags(r.b, st, cudaEventRecordExternal);
+            trace_record(r.b, st);
             c->rec->push_back(r);
         }
     }
@@ -512,6 +526,7 @@ TileArgs stack_tile_args(const fi_ctx* c, long long n) {
     TileArgs a;
     memset(&a, 0, sizeof(a));
     a.act = c->act;
+    a.act_out = c->yout ? c->yout : c->act + c->G * c->L;
     a.h = c->h;
     a.L = c->L;
     a.G = c->G;
@@ -528,18 +543,37 @@ TileArgs stack_tile_args(const fi_ctx* c, long long n) {
 // The gray blocks of every layer released after the n-th token, one launch
 // (section "Schicht-uebergreifende Parallelisierung (Algorithmus 3)").
 int launch_block(fi_ctx* c, long long n, int impl, cudaStream_t st, int pdl = 0, int force_acc = 0,
-                 const TokIO* io = nullptr) {
+                 TokIO* io = nullptr) {
     TileArgs a = stack_tile_args(c, n);
     if (force_acc) a.overwrite = 0;
     a.io = io;  // replayed per-token graph: the kernels take n from the step record
+    a.advance = io ? 1 : 0;  // and this launch closes the token
     const int q = ctz64(n);
     const int cls = impl == FI_TAU_DIRECT ? FI_K_BLOCK_DIRECT
                     : (q <= fused_qmax() ? FI_K_BLOCK_FFT : FI_K_BLOCK_CLUSTER);
-    LaunchScope scope(c, cls, st, q);
-    if (impl == FI_TAU_DIRECT) return launch_direct_tile(a, st);
-    a.spec = c->spec[q];
-    a.spec_stride = c->spec_stride[q];
-    return launch_fft(q, a, st, pdl);
+    if (impl != FI_TAU_DIRECT) {
+        a.spec = c->spec[q];
+        a.spec_stride = c->spec_stride[q];
+    }
+    auto one = [&](const TileArgs& b) {
+        LaunchScope scope(c, cls, st, q);
+        return impl == FI_TAU_DIRECT ? launch_direct_tile(b, st) : launch_fft(q, b, st, pdl);
+    };
+    if (!c->layer_split) return one(a);
+    // ablation: the same blocks as M launches of one layer each (the layer's buffers,
+    // filters and spectra addressed as layer 0 of a one-layer stack)
+    for (int l = 0; l < c->M; ++l) {
+        TileArgs b = a;
+        b.act = a.act + (long long)l * c->G * c->L;
+        b.act_out = a.act_out + (long long)l * c->G * c->L;
+        b.h = a.h + (long long)l * c->D * c->L;
+        if (b.spec) b.spec = a.spec + (long long)l * c->D * a.spec_stride;
+        b.count = (int)c->G;
+        b.advance = (l == c->M - 1) ? a.advance : 0;  // only the last launch closes the token
+        int rc = one(b);
+        if (rc) return rc;
+    }
+    return FI_OK;
 }
 
 int upload_twiddles(fi_ctx* c) {
@@ -699,9 +733,10 @@ int tau_of(const fi_ctx* c, int q) { return c->tau_user[q] ? c->tau_user[q] : c-
 
 // ---------------------------------------------------------------- launch sequences
 int enqueue_token(fi_ctx* c, long long t, const float* x, float* y, int closed, cudaStream_t st,
-                  const TokIO* io = nullptr) {
+                  TokIO* io = nullptr) {
     StepArgs a;
     a.io = io;
+    a.advance = 0;
     a.act = c->act;
     a.h = c->h;
     a.M = c->M;
@@ -721,27 +756,25 @@ int enqueue_token(fi_ctx* c, long long t, const float* x, float* y, int closed, 
         if (q <= kFuseQMax && impl == FI_TAU_DIRECT) a.fuseU = 1 << q;
     }
     const int grid = (int)((c->G + 31) / 32);
+    const bool block_follows = n < c->L && a.fuseU == 0;
+    a.advance = (io && !block_follows) ? 1 : 0;  // the step kernel closes the token itself
     {
         LaunchScope scope(c, FI_K_TOKEN_STEP, st);
         k_token_step<kStepNT><<<grid, kStepNT, 0, st>>>(a);
         CK(cudaGetLastError());
     }
-    if (n < c->L && a.fuseU == 0) return launch_block(c, n, impl, st, 0, 0, io);
+    if (block_follows) return launch_block(c, n, impl, st, 0, 0, io);
     return FI_OK;
 }
 
 // The launches of one token step with the token taken from the step record: the step
-// kernel, the block released after it (edge 2^q; none for the last token), and the
-// advance of the record.  Captured once per (mode, q) into a graph.
+// kernel and the block released after it (edge 2^q; none for the last token), the last
+// of them advancing the record.  Captured once per (mode, q) into a graph.
 int capture_token_graph(fi_ctx* c, int closed, int idx) {
     const long long t = idx == 32 ? c->L - 1 : (1LL << idx) - 1;  // a token releasing edge 2^idx
     c->enq_launches = 0;
     CK(cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed));
     int rc = enqueue_token(c, t, nullptr, nullptr, closed, c->cap, c->tio);
-    if (!rc) {
-        k_advance_step<<<1, 1, 0, c->cap>>>(c->tio);
-        c->enq_launches++;
-    }
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(c->cap, &graph);
     if (!rc && e == cudaSuccess) e = cudaGetLastError();
@@ -782,6 +815,7 @@ int run_token_graphs(fi_ctx* c, long long t0, long long steps, const float* x, f
     v.tx = t0;
     v.t = t0;
     v.closed = closed;
+    v.done = 0;
     k_set_step<<<1, 1, 0, c->stream>>>(c->tio, v);
     CK(cudaGetLastError());
     long long nl = 1;
@@ -860,7 +894,8 @@ void drop_graphs(fi_ctx* c) {
 // "Implementierungsdetails": CUDA graphs remove the per-launch CPU overhead).
 // The Lazy / Eager baselines: one launch per token, one CTA per chain.
 int run_baseline(fi_ctx* c, long long t0, long long steps, const float* x, float* out, int closed) {
-    const bool eager = c->path == FI_PATH_EAGER;
+    const bool eager = c->path == FI_PATH_EAGER || c->path == FI_PATH_EAGER_NP;
+    const bool np = c->path == FI_PATH_LAZY_NP || c->path == FI_PATH_EAGER_NP;
     if (eager && t0 == 0)  // running sums of layers 1..M start at zero
         CK(cudaMemsetAsync(c->act + c->G * c->L, 0, sizeof(float) * c->M * c->G * c->L, c->stream));
     BaseArgs a;
@@ -874,16 +909,27 @@ int run_baseline(fi_ctx* c, long long t0, long long steps, const float* x, float
     a.x = x;
     a.out = out;
     a.closed = closed;
-    const int threads = eager ? 512 : 32 * std::min(c->M, 32);
+    const int threads = 32 * std::min(c->M, 32);
     const size_t smem = (size_t)(2 * c->M + 1) * sizeof(float);
+    const int np_threads = eager ? 512 : 256;
     for (long long t = t0; t < t0 + steps; ++t) {
         a.t = t;
         a.first = t == t0;
-        if (eager) k_eager_token<<<(unsigned)c->G, threads, smem, c->stream>>>(a);
-        else k_lazy_token<<<(unsigned)c->G, threads, smem, c->stream>>>(a);
+        if (np) {
+            // one launch per layer, in layer order: no two layers' work side by side
+            for (int l = 1; l <= c->M; ++l) {
+                if (eager) k_eager_layer<<<(unsigned)c->G, np_threads, 0, c->stream>>>(a, l);
+                else k_lazy_layer<<<(unsigned)c->G, np_threads, (np_threads / 32) * sizeof(float), c->stream>>>(a, l);
+            }
+        } else if (eager) {
+            k_eager_chain<<<(unsigned)((c->G + 127) / 128), 128, 0, c->stream>>>(a);
+            k_eager_push<<<dim3((unsigned)c->G, (unsigned)c->M), 256, 0, c->stream>>>(a);
+        } else {
+            k_lazy_token<<<(unsigned)c->G, threads, smem, c->stream>>>(a);
+        }
     }
     CK(cudaGetLastError());
-    c->launches += steps;
+    c->launches += np ? steps * c->M : (eager ? 2 * steps : steps);
     c->last_trace = nullptr;
     return FI_OK;
 }
@@ -1077,6 +1123,7 @@ int create_impl(fi_ctx* c, const float* filters) {
     CK(cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev));
     CK(cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking));
     if (const char* e = getenv("FI_PDL")) c->pdl = atoi(e) ? 1 : 0;
+    if (const char* e = getenv("FI_LAYER_SPLIT")) c->layer_split = atoi(e) ? 1 : 0;
     const long long M = c->M, D = c->D, L = c->L, G = c->G;
     int rc;
     if ((rc = dev_alloc(c, &c->act, (size_t)(M + 1) * G * L))) return rc;
@@ -1178,6 +1225,276 @@ int prefill_impl(fi_ctx* c, const float* x, int p, float* y) {
     c->last_trace = nullptr;
     return FI_OK;
 }
+
+// ====================================================================== language model
+// The Hyena-like model around the mixer (fi_lm.cuh has the layer it computes): one
+// mixer context holds the long convolutions (act = the mixer inputs x of every layer,
+// yout = their outputs y, filters and spectra), the rest are bf16 weights and small
+// per-token buffers.  A token is a host-issued launch sequence: embedding; per layer
+// the in-projection, the mixer step, the MLP; the LM head and the greedy choice; then
+// the gray blocks of every layer in one launch (section "Schicht-uebergreifende
+// Parallelisierung (Algorithmus 3)").
+constexpr unsigned kLmMagic = 0xF1C71A11u;
+
+struct fi_lm {
+    unsigned magic = kLmMagic;
+    fi_ctx* mix = nullptr;
+    int M = 0, B = 0, D = 0, L = 0, V = 0;
+    long long t = 0;
+    __nv_bfloat16 *E = nullptr, *Wlm = nullptr, *Win = nullptr, *W1 = nullptr, *W2 = nullptr;
+    float* conv = nullptr;                       // [M][3][3D]
+    float *u = nullptr, *z = nullptr, *zr = nullptr, *m1 = nullptr, *logits = nullptr;
+    int *tok = nullptr, *next = nullptr;         // [B]: the next input token, the latest choice
+    int* stage_i = nullptr;                      // host token arrays staged on the device
+    size_t stage_i_n = 0;
+    float* stage_f = nullptr;
+    size_t stage_f_n = 0;
+    // tracing: events around the mixer's block launches (every token) and mixer steps
+    // (every kTraceEvery-th token), and around each whole call
+    int trace_on = 0;
+    std::vector<cudaEvent_t> ev;
+    std::vector<std::pair<int, int>> ev_blocks, ev_steps;  // event index pairs
+    int ev_call0 = -1, ev_call1 = -1;
+    long long traced_tokens = 0, sampled_tokens = 0;
+};
+
+namespace {
+
+std::mutex g_lm_mu;
+std::set<const fi_lm*> g_lm_live;
+constexpr int kTraceEvery = 64;
+
+int check_lm(const fi_lm* m) {
+    std::lock_guard<std::mutex> lk(g_lm_mu);
+    if (!m || !g_lm_live.count(m) || m->magic != kLmMagic) return set_err(FI_ESTATE, "null or destroyed model");
+    return FI_OK;
+}
+
+template <typename T>
+int lm_alloc(fi_lm* m, T** p, size_t count) {
+    return dev_alloc(m->mix, p, count);
+}
+
+// fp32 host or device weights -> bf16 device array
+int lm_upload_bf16(fi_lm* m, const float* src, size_t n, __nv_bfloat16** dst) {
+    int rc = lm_alloc(m, dst, n);
+    if (rc) return rc;
+    float* tmp = nullptr;
+    CK(cudaMalloc((void**)&tmp, n * sizeof(float)));
+    cudaError_t e = cudaMemcpy(tmp, src, n * sizeof(float), cudaMemcpyDefault);
+    if (e == cudaSuccess) {
+        k_to_bf16<<<1184, 256>>>(tmp, (long long)n, *dst);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    cudaFree(tmp);
+    if (e != cudaSuccess) return set_err(FI_ECUDA, "weight upload failed: %s", cudaGetErrorString(e));
+    return FI_OK;
+}
+
+int lm_event(fi_lm* m, cudaStream_t st) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    cudaEventRecord(e, st);
+    m->ev.push_back(e);
+    return (int)m->ev.size() - 1;
+}
+
+void lm_clear_trace(fi_lm* m) {
+    for (cudaEvent_t e : m->ev) cudaEventDestroy(e);
+    m->ev.clear();
+    m->ev_blocks.clear();
+    m->ev_steps.clear();
+    m->ev_call0 = m->ev_call1 = -1;
+    m->traced_tokens = m->sampled_tokens = 0;
+}
+
+template <int EPI>
+int lm_gemv(const __nv_bfloat16* W, int N, int K, const float* x, int B, int ln, float* y, cudaStream_t st) {
+    const int rows_per_cta = kLmThreads / 32;
+    const int grid = std::min((N + rows_per_cta - 1) / rows_per_cta, 8 * 148);
+    k_lm_gemv<EPI><<<grid, kLmThreads, (size_t)B * K * sizeof(float), st>>>(W, N, K, x, B, ln, y);
+    CK(cudaGetLastError());
+    return FI_OK;
+}
+
+// One token t: tok_src [B] (device) is its input; logits_out [B][V] (device) or null;
+// next_out [B] (device) receives the greedy choice, also kept as the next input.
+int lm_token(fi_lm* m, long long t, const int* tok_src, float* logits_out, int* next_out, cudaStream_t st) {
+    const int M = m->M, B = m->B, D = m->D, V = m->V;
+    const long long L = m->L, G = (long long)B * D;
+    fi_ctx* c = m->mix;
+    int rc;
+    k_lm_embed<<<(B * D + 255) / 256, 256, 0, st>>>(m->E, tok_src, B, D, m->u);
+    const bool sample = m->trace_on && (t % kTraceEvery == 0);
+    for (int l = 0; l < M; ++l) {
+        if ((rc = lm_gemv<kLmStore>(m->Win + (size_t)l * 3 * D * D, 3 * D, D, m->u, B, 1, m->z, st))) return rc;
+        const int e0 = sample ? lm_event(m, st) : -1;
+        k_lm_mixer<<<(B * D + 127) / 128, 128, 0, st>>>(m->z, m->zr + (size_t)l * 2 * B * 3 * D,
+                                                       m->conv + (size_t)l * 9 * D, c->h + (size_t)l * D * L, L, B,
+                                                       D, t, c->act + (size_t)l * G * L, c->yout + (size_t)l * G * L,
+                                                       m->u);
+        if (sample) m->ev_steps.push_back({e0, lm_event(m, st)});
+        CK(cudaGetLastError());
+        if ((rc = lm_gemv<kLmGelu>(m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->u, B, 1, m->m1, st))) return rc;
+        if ((rc = lm_gemv<kLmAdd>(m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, st))) return rc;
+    }
+    float* lg = logits_out ? logits_out : m->logits;
+    if ((rc = lm_gemv<kLmStore>(m->Wlm, V, D, m->u, B, 1, lg, st))) return rc;
+    k_lm_argmax<<<B, 256, 0, st>>>(lg, V, m->tok, next_out);
+    CK(cudaGetLastError());
+    if (t + 1 < L) {
+        const int e0 = m->trace_on ? lm_event(m, st) : -1;
+        if ((rc = launch_block(c, t + 1, tau_of(c, ctz64(t + 1)), st))) return rc;
+        if (m->trace_on) m->ev_blocks.push_back({e0, lm_event(m, st)});
+    }
+    if (m->trace_on) {
+        m->traced_tokens++;
+        if (sample) m->sampled_tokens++;
+    }
+    return FI_OK;
+}
+
+int lm_stage(fi_lm* m, const int* src, size_t n, const int** out) {
+    if (is_device_ptr(src)) {
+        *out = src;
+        return FI_OK;
+    }
+    if (m->stage_i_n < n) {
+        cudaFree(m->stage_i);
+        m->stage_i = nullptr;
+        m->stage_i_n = 0;
+        int rc = lm_alloc(m, &m->stage_i, n);
+        if (rc) return rc;
+        m->stage_i_n = n;
+    }
+    CK(cudaMemcpyAsync(m->stage_i, src, n * sizeof(int), cudaMemcpyHostToDevice, m->mix->stream));
+    *out = m->stage_i;
+    return FI_OK;
+}
+
+// a run of tokens: teacher (tokens [steps][B]) or closed loop (tok0 [B] at t = 0, or
+// continuing from the last choice); outputs logits [steps][B][V] (or null) and the
+// greedy choices [steps][B]
+int lm_run(fi_lm* m, const int* tokens, const int* tok0, int steps, float* logits, int* next) {
+    if (steps < 0) return set_err(FI_EINVAL, "steps must be >= 0");
+    if (m->t + steps > m->L) return set_err(FI_ECAPACITY, "t=%lld + steps=%d exceeds capacity L=%d", m->t, steps, m->L);
+    if (steps == 0) return FI_OK;
+    if (!next) return set_err(FI_EINVAL, "the output token array is NULL");
+    cudaStream_t st = m->mix->stream;
+    const int B = m->B, V = m->V;
+    int rc;
+    const int* tok_d = nullptr;
+    if (tokens) {
+        if ((rc = lm_stage(m, tokens, (size_t)steps * B, &tok_d))) return rc;
+    } else if (tok0) {
+        const int* t0d = nullptr;
+        if ((rc = lm_stage(m, tok0, (size_t)B, &t0d))) return rc;
+        CK(cudaMemcpyAsync(m->tok, t0d, B * sizeof(int), cudaMemcpyDeviceToDevice, st));
+    } else if (m->t == 0) {
+        return set_err(FI_EINVAL, "closed loop at t=0 needs the start tokens");
+    }
+    const bool n_host = !is_device_ptr(next);
+    const bool l_host = logits && !is_device_ptr(logits);
+    int* next_d = next;
+    float* logits_d = logits;
+    const size_t need_f = (n_host ? (size_t)steps * B : 0) + (l_host ? (size_t)steps * B * V : 0);
+    if (need_f > m->stage_f_n) {
+        cudaFree(m->stage_f);
+        m->stage_f = nullptr;
+        m->stage_f_n = 0;
+        if ((rc = lm_alloc(m, &m->stage_f, need_f))) return rc;
+        m->stage_f_n = need_f;
+    }
+    if (n_host) next_d = reinterpret_cast<int*>(m->stage_f);
+    if (l_host) logits_d = m->stage_f + (n_host ? (size_t)steps * B : 0);
+    if (m->t == 0) CK(cudaMemsetAsync(m->zr, 0, sizeof(float) * (size_t)m->M * 2 * B * 3 * m->D, st));
+    if (m->trace_on) {
+        lm_clear_trace(m);
+        m->ev_call0 = lm_event(m, st);
+    }
+    for (int k = 0; k < steps; ++k) {
+        const int* src = tokens ? tok_d + (size_t)k * B : m->tok;
+        if ((rc = lm_token(m, m->t + k, src, logits ? logits_d + (size_t)k * B * V : nullptr,
+                           next_d + (size_t)k * B, st)))
+            return rc;
+    }
+    if (m->trace_on) m->ev_call1 = lm_event(m, st);
+    m->t += steps;
+    if (n_host) CK(cudaMemcpyAsync(next, next_d, sizeof(int) * steps * B, cudaMemcpyDeviceToHost, st));
+    if (l_host) CK(cudaMemcpyAsync(logits, logits_d, sizeof(float) * steps * B * V, cudaMemcpyDeviceToHost, st));
+    if (n_host || l_host) CK(cudaStreamSynchronize(st));
+    return FI_OK;
+}
+
+void lm_free(fi_lm* m) {
+    if (!m) return;
+    lm_clear_trace(m);
+    if (m->mix) {
+        cudaStreamSynchronize(m->mix->stream);
+        cudaFree(m->mix->yout);
+        m->mix->yout = nullptr;
+        free_ctx(m->mix);
+    }
+    cudaFree(m->E);
+    cudaFree(m->Wlm);
+    cudaFree(m->Win);
+    cudaFree(m->W1);
+    cudaFree(m->W2);
+    cudaFree(m->conv);
+    cudaFree(m->u);
+    cudaFree(m->z);
+    cudaFree(m->zr);
+    cudaFree(m->m1);
+    cudaFree(m->logits);
+    cudaFree(m->tok);
+    cudaFree(m->next);
+    cudaFree(m->stage_i);
+    cudaFree(m->stage_f);
+    m->magic = 0;
+    delete m;
+}
+
+int lm_create_impl(fi_lm* m, const float* E, const float* Wlm, const float* Win, const float* conv,
+                   const float* W1, const float* W2, const float* filters) {
+    const int M = m->M, B = m->B, D = m->D, V = m->V;
+    fi_ctx* c = new fi_ctx();
+    m->mix = c;
+    c->M = M;
+    c->B = B;
+    c->D = D;
+    c->L = m->L;
+    c->G = (long long)B * D;
+    while ((1 << c->P) < c->L) ++c->P;
+    int rc = create_impl(c, filters);
+    if (rc) return rc;
+    if ((rc = dev_alloc(c, &c->yout, (size_t)M * c->G * c->L))) return rc;
+    CK(cudaFuncSetAttribute(k_lm_gemv<kLmStore>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax - 1024));
+    CK(cudaFuncSetAttribute(k_lm_gemv<kLmGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax - 1024));
+    CK(cudaFuncSetAttribute(k_lm_gemv<kLmAdd>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax - 1024));
+    const size_t DD = (size_t)D * D;
+    if ((rc = lm_upload_bf16(m, E, (size_t)V * D, &m->E))) return rc;
+    if ((rc = lm_upload_bf16(m, Wlm, (size_t)V * D, &m->Wlm))) return rc;
+    if ((rc = lm_upload_bf16(m, Win, (size_t)M * 3 * DD, &m->Win))) return rc;
+    if ((rc = lm_upload_bf16(m, W1, (size_t)M * 4 * DD, &m->W1))) return rc;
+    if ((rc = lm_upload_bf16(m, W2, (size_t)M * 4 * DD, &m->W2))) return rc;
+    if ((rc = lm_alloc(m, &m->conv, (size_t)M * 9 * D))) return rc;
+    CK(cudaMemcpy(m->conv, conv, sizeof(float) * M * 9 * D, cudaMemcpyDefault));
+    if ((rc = lm_alloc(m, &m->u, (size_t)B * D))) return rc;
+    if ((rc = lm_alloc(m, &m->z, (size_t)B * 3 * D))) return rc;
+    if ((rc = lm_alloc(m, &m->zr, (size_t)M * 2 * B * 3 * D))) return rc;
+    if ((rc = lm_alloc(m, &m->m1, (size_t)B * 4 * D))) return rc;
+    if ((rc = lm_alloc(m, &m->logits, (size_t)B * V))) return rc;
+    if ((rc = lm_alloc(m, &m->tok, (size_t)B))) return rc;
+    if ((rc = lm_alloc(m, &m->next, (size_t)B))) return rc;
+    CK(cudaDeviceSynchronize());
+    return FI_OK;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -1356,12 +1673,14 @@ int fi_set_stream(fi_ctx* ctx, void* stream) {
 int fi_set_path(fi_ctx* ctx, int path) {
     int rc = check_ctx(ctx);
     if (rc) return rc;
-    if (path < FI_PATH_WINDOW || path > FI_PATH_EAGER) return set_err(FI_EINVAL, "unknown path %d", path);
+    if (path < FI_PATH_WINDOW || path > FI_PATH_EAGER_NP) return set_err(FI_EINVAL, "unknown path %d", path);
     if (path == FI_PATH_WINDOW && ctx->W == 0)
         return set_err(FI_EINVAL, "window path unavailable for this shape (shared memory)");
     const bool base_new = path >= FI_PATH_LAZY, base_old = ctx->path >= FI_PATH_LAZY;
     if (path != ctx->path && ctx->t != 0 && (base_new || base_old))
         return set_err(FI_EINVAL, "the lazy and eager paths keep their own state: switch to or from them at t = 0");
+    if (base_new && base_old && path != ctx->path && ctx->t != 0)
+        return set_err(FI_EINVAL, "switch between the baselines at t = 0");
     ctx->path = path;
     return FI_OK;
 }
@@ -1399,7 +1718,8 @@ int fi_get_info(const fi_ctx* ctx, fi_info* info) {
     info->t = (int)ctx->t;
     info->window = ctx->W;
     info->chains_per_cta = ctx->kch * ctx->B;
-    info->path = (ctx->path == FI_PATH_WINDOW && ctx->W) ? FI_PATH_WINDOW : FI_PATH_TOKEN;
+    info->path = ctx->path >= FI_PATH_LAZY ? ctx->path
+                 : ((ctx->path == FI_PATH_WINDOW && ctx->W) ? FI_PATH_WINDOW : FI_PATH_TOKEN);
     info->graphs = ctx->graphs;
     for (int q = 0; q < ctx->P && q < 32; ++q) {
         info->tau[q] = tau_of(ctx, q);
@@ -1440,6 +1760,25 @@ int fi_trace_read(fi_ctx* ctx, fi_trace* out) {
         }
     }
     return FI_OK;
+}
+
+int fi_trace_launches(fi_ctx* ctx, int max, int* cls, int* q, float* us) {
+    int rc = check_ctx(ctx);
+    if (rc) return rc;
+    if (max < 0 || (max > 0 && (!cls || !q || !us)))
+        return set_err(FI_EINVAL, "fi_trace_launches: need max >= 0 and non-NULL arrays");
+    if (!ctx->last_trace) return 0;
+    CK(cudaStreamSynchronize(ctx->stream));
+    const int n = (int)ctx->last_trace->size();
+    for (int i = 0; i < n && i < max; ++i) {
+        const TraceRec& r = (*ctx->last_trace)[i];
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, r.a, r.b));
+        cls[i] = r.cls;
+        q[i] = r.q;
+        us[i] = 1000.f * ms;
+    }
+    return n;
 }
 
 int fi_debug_schedule(const fi_ctx* ctx, int n, int* U, int* impl, int* src_lo, int* dst_lo, int* dst_hi) {
@@ -1494,6 +1833,102 @@ int fi_tau_fft_noalloc(int U, int count, const float* blocks, const float* taps,
     int rc = set_all_attrs();
     if (rc) return rc;
     return tau_fft_noalloc_impl(U, q, count, blocks, taps, ldt, out, accumulate);
+}
+
+
+// ---------------------------------------------------------------- language model
+fi_lm* fi_lm_create(int layers, int B, int D, int L, int V, const float* E, const float* W_lm, const float* W_in,
+                    const float* conv, const float* W1, const float* W2, const float* filters) {
+    g_err[0] = 0;
+    if (layers < 1 || B < 1 || B > kLmMaxB || D < 8 || (D % 8) || L < 2 || (L & (L - 1)) || V < 1 || !E ||
+        !W_lm || !W_in || !conv || !W1 || !W2 || !filters) {
+        set_err(FI_EINVAL, "fi_lm_create: need layers >= 1, 1 <= B <= %d, D a multiple of 8, L a power of two "
+                           ">= 2, V >= 1 and non-NULL weights", kLmMaxB);
+        return nullptr;
+    }
+    if (L > (1 << (kFftQMax + 1))) {
+        set_err(FI_EINVAL, "fi_lm_create: L = %d above %d", L, 1 << (kFftQMax + 1));
+        return nullptr;
+    }
+    fi_lm* m = new fi_lm();
+    m->M = layers;
+    m->B = B;
+    m->D = D;
+    m->L = L;
+    m->V = V;
+    int rc = lm_create_impl(m, E, W_lm, W_in, conv, W1, W2, filters);
+    if (rc) {
+        std::string msg = g_err;
+        lm_free(m);
+        cudaGetLastError();
+        set_err(rc, "%s", msg.c_str());
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_lm_mu);
+    g_lm_live.insert(m);
+    return m;
+}
+
+void fi_lm_destroy(fi_lm* m) {
+    {
+        std::lock_guard<std::mutex> lk(g_lm_mu);
+        if (!m || !g_lm_live.count(m)) return;
+        g_lm_live.erase(m);
+    }
+    lm_free(m);
+}
+
+int fi_lm_reset(fi_lm* m) {
+    int rc = check_lm(m);
+    if (rc) return rc;
+    m->t = 0;
+    m->mix->t = 0;
+    return FI_OK;
+}
+
+int fi_lm_forward(fi_lm* m, const int* tokens, int steps, float* logits, int* next) {
+    int rc = check_lm(m);
+    if (rc) return rc;
+    if (!tokens && steps > 0) return set_err(FI_EINVAL, "fi_lm_forward: tokens is NULL");
+    return lm_run(m, tokens, nullptr, steps, logits, next);
+}
+
+int fi_lm_generate(fi_lm* m, const int* tok0, int steps, int* next) {
+    int rc = check_lm(m);
+    if (rc) return rc;
+    return lm_run(m, nullptr, tok0, steps, nullptr, next);
+}
+
+int fi_lm_set_trace(fi_lm* m, int on) {
+    int rc = check_lm(m);
+    if (rc) return rc;
+    m->trace_on = on ? 1 : 0;
+    if (!on) lm_clear_trace(m);
+    return FI_OK;
+}
+
+int fi_lm_split(fi_lm* m, double* mixer_us, double* total_us) {
+    int rc = check_lm(m);
+    if (rc) return rc;
+    if (!mixer_us || !total_us) return set_err(FI_EINVAL, "fi_lm_split: NULL output");
+    *mixer_us = *total_us = 0.0;
+    if (m->ev_call0 < 0 || m->ev_call1 < 0) return FI_OK;
+    CK(cudaStreamSynchronize(m->mix->stream));
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, m->ev[m->ev_call0], m->ev[m->ev_call1]));
+    *total_us = 1000.0 * ms;
+    double blocks = 0.0, steps = 0.0;
+    for (auto& pr : m->ev_blocks) {
+        CK(cudaEventElapsedTime(&ms, m->ev[pr.first], m->ev[pr.second]));
+        blocks += 1000.0 * ms;
+    }
+    for (auto& pr : m->ev_steps) {
+        CK(cudaEventElapsedTime(&ms, m->ev[pr.first], m->ev[pr.second]));
+        steps += 1000.0 * ms;
+    }
+    const double scale = m->sampled_tokens ? (double)m->traced_tokens / (double)m->sampled_tokens : 0.0;
+    *mixer_us = blocks + steps * scale;
+    return FI_OK;
 }
 
 }  // extern "C"

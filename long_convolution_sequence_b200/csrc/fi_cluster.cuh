@@ -53,15 +53,19 @@ __device__ __forceinline__ void cluster_forward(const float2* __restrict__ z, fl
     // y[n2] = W_N^{n2 k1} sum_{n1} z[n1 N2 + n2] W_NC^{n1 k1}, n2 = b + r NB: the twiddle
     // is W_N^{b k1} (one table entry per butterfly) times W_N^{r NB k1} (the same for
     // every thread of the CTA)
-    auto y_at = [&](int b, int r, int NB, float2 wb) {
-        const int n2 = b + r * NB;
-        float2 y = __ldg(z + n2);
+    auto y_of = [&](const float2 (&zz)[NIN], int r, int NB, float2 wb) {
+        float2 y = zz[0];
 #pragma unroll
-        for (int n1 = 1; n1 < NIN; ++n1) {
-            const float2 zz = __ldg(z + n1 * N2 + n2);
-            y = make_float2(y.x + (zz.x * wn1[n1].x - zz.y * wn1[n1].y), y.y + (zz.x * wn1[n1].y + zz.y * wn1[n1].x));
-        }
+        for (int n1 = 1; n1 < NIN; ++n1)
+            y = make_float2(y.x + (zz[n1].x * wn1[n1].x - zz[n1].y * wn1[n1].y),
+                            y.y + (zz[n1].x * wn1[n1].y + zz[n1].y * wn1[n1].x));
         return fft::cm(y, fft::cm(wb, fft::tw_at<TWLOG>(tw, (r * NB * k1) << (TWLOG - LOGN))));
+    };
+    auto y_at = [&](int b, int r, int NB, float2 wb) {
+        float2 zz[NIN];
+#pragma unroll
+        for (int n1 = 0; n1 < NIN; ++n1) zz[n1] = __ldg(z + n1 * N2 + b + r * NB);
+        return y_of(zz, r, NB, wb);
     };
     if constexpr (R0 > 1) {
         // radix-R0 first pass (Ns = 1): butterfly b reads y[b + r N2/R0]
@@ -83,8 +87,19 @@ __device__ __forceinline__ void cluster_forward(const float2* __restrict__ z, fl
     } else {
         constexpr int NB = N2 / 16;
         const float2 wb = fft::tw_at<TWLOG>(tw, (t * k1) << (TWLOG - LOGN));
+        // the inputs of RB outputs are loaded before any is combined: the loads of a
+        // batch are in flight together (the sums are bound by global-memory latency)
+        constexpr int RB = NIN >= 32 ? 1 : (32 / NIN > 16 ? 16 : 32 / NIN);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) v[0][r] = y_at(t, r, NB, wb);
+        for (int r0 = 0; r0 < 16; r0 += RB) {
+            float2 zz[RB][NIN];
+#pragma unroll
+            for (int i = 0; i < RB; ++i)
+#pragma unroll
+                for (int n1 = 0; n1 < NIN; ++n1) zz[i][n1] = __ldg(z + n1 * N2 + t + (r0 + i) * NB);
+#pragma unroll
+            for (int i = 0; i < RB; ++i) v[0][r0 + i] = y_of(zz[i], r0 + i, NB, wb);
+        }
         fft::dft<16>(v[0]);
 #pragma unroll
         for (int m = 0; m < 16; ++m) X[fft::pad(t * 16 + m)] = v[0][fft::omap<16>(m)];
@@ -170,13 +185,18 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
             q[m] = r;
         }
     }
-    cluster.sync();  // partner reads done before X is overwritten; Hs is free
+    // The inverse runs in the spectrum area, free once this CTA's threads have read it:
+    // X keeps this CTA's Z, which the partner CTA may still be reading, so no cluster
+    // barrier is needed here.
+    __syncthreads();
     grid_dep_launch();
+    float2* X2 = Hs;
     // this CTA's old outputs (runs [k1 PER, (k1+1) PER) + N2 i, i < NC/2) stream into
-    // the spectrum area during the inverse transform
+    // the rest of the spectrum area during the inverse transform
     constexpr int PER = N2 / NC;  // output n2 values of this CTA
     static_assert(PER % T == 0, "outputs per CTA must be a multiple of its threads");
-    float2* Os = Hs;
+    static_assert(G::SME + N2 / 2 <= G::HST, "inverse area and old outputs fit the spectrum area");
+    float2* Os = Hs + G::SME;
     if (!a.overwrite) {
         const float2* o2c = reinterpret_cast<const float2*>(p.out);
 #pragma unroll
@@ -188,14 +208,14 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
     // ---- inverse, local N2-point DFT over k2: first pass in registers (Ns = 1)
     fft::dft<16>(q);
 #pragma unroll
-    for (int m = 0; m < 16; ++m) X[fft::pad(t * 16 + m)] = q[fft::omap<16>(m)];
+    for (int m = 0; m < 16; ++m) X2[fft::pad(t * 16 + m)] = q[fft::omap<16>(m)];
     __syncthreads();
     // remaining passes; the last one multiplies its outputs n2 by W_N^{k1 n2} and
     // leaves them in natural order
     {
         constexpr int NLAST = R0 > 1 ? NP : NP - 1;  // radix-16 passes after the first
 #pragma unroll
-        for (int j = 1; j < NLAST; ++j) fft::pass<LOGN2, 16, 1, TWLOG>(X, v, t, T, 4 * j, a.tw);
+        for (int j = 1; j < NLAST; ++j) fft::pass<LOGN2, 16, 1, TWLOG>(X2, v, t, T, 4 * j, a.tw);
         if constexpr (R0 > 1) {
             // radix-R0 at Ns = N2/R0: butterfly b (< N2/R0) reads X[b + r N2/R0]
             constexpr int BPT = 16 / R0, NB = N2 / R0;
@@ -204,7 +224,7 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
             for (int u = 0; u < BPT; ++u) {
                 const int b = t + u * T;
 #pragma unroll
-                for (int r = 0; r < R0; ++r) w[u][r] = X[fft::pad(b + r * NB)];
+                for (int r = 0; r < R0; ++r) w[u][r] = X2[fft::pad(b + r * NB)];
                 fft::apply_twiddles<R0, TWLOG>(w[u], a.tw, LOGN2, b);
                 fft::dft<R0>(w[u]);
             }
@@ -216,7 +236,7 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
 #pragma unroll
                 for (int m = 0; m < R0; ++m) {
                     const float2 wm = fft::cm(wb, fft::tw_at<TWLOG>(a.tw, (m * NB * k1) << (TWLOG - LOGN)));
-                    X[fft::pad(b + m * NB)] = fft::cm(w[u][fft::omap<R0>(m)], wm);
+                    X2[fft::pad(b + m * NB)] = fft::cm(w[u][fft::omap<R0>(m)], wm);
                 }
             }
         } else {
@@ -224,7 +244,7 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
             constexpr int NB = N2 / 16;
             float2 w[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) w[r] = X[fft::pad(t + r * NB)];
+            for (int r = 0; r < 16; ++r) w[r] = X2[fft::pad(t + r * NB)];
             fft::apply_twiddles<16, TWLOG>(w, a.tw, LOGN2, t);
             fft::dft<16>(w);
             __syncthreads();
@@ -232,7 +252,7 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
                 const float2 wm = fft::cm(wb, fft::tw_at<TWLOG>(a.tw, (m * NB * k1) << (TWLOG - LOGN)));
-                X[fft::pad(t + m * NB)] = fft::cm(w[fft::omap<16>(m)], wm);
+                X2[fft::pad(t + m * NB)] = fft::cm(w[fft::omap<16>(m)], wm);
             }
         }
     }
@@ -247,10 +267,13 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
         float2 g[NPT][NC];
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-            const float2* Xc = cluster.map_shared_rank(X, c);
+            const float2* Xc = cluster.map_shared_rank(X2, c);
 #pragma unroll
             for (int u = 0; u < NPT; ++u) g[u][c] = Xc[fft::pad(k1 * PER + t + u * T)];
         }
+        // this CTA's reads of the others' shared memory are done (release); the wait,
+        // before exit, overlaps the output stores
+        asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
 #pragma unroll
         for (int u = 0; u < NPT; ++u) {
             const int j = t + u * T;
@@ -269,7 +292,8 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
             }
         }
     }
-    cluster.sync();  // no CTA leaves while another still reads its shared memory
+    asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");  // no CTA leaves while another reads it
+    if (a.io && a.advance) tok_advance_if_last(a.io);
 }
 
 // Spectra of the cluster sizes: H = scale * DFT_{2N}(taps[0, 2N)), k = 0..N, in CTA

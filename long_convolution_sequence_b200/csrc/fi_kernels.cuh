@@ -90,23 +90,41 @@ __device__ __forceinline__ float2 conjf2(float2 a) { return make_float2(a.x, -a.
 // "Implementierungsdetails": the launches of one token step are recorded once and
 // replayed), so the token a replay works on cannot be a kernel argument: it lives in
 // this device-side record, written by k_set_step at the start of a call and advanced
-// by k_advance_step at the end of every token.
+// by the last CTA to finish the token's last launch (tok_advance_if_last).
 struct TokIO {
     const float* x;  // teacher: tokens [.][G] from token tx on; closed loop: [G] token tx, or null
     float* y;        // y^M [.][G] from token tx on
     long long tx;    // token of x[0] / y[0]
     long long t;     // token being processed
     int closed;
+    unsigned done;   // CTAs of the current launch that have finished (advancing launch only)
 };
 
 __global__ void k_set_step(TokIO* io, TokIO v) { *io = v; }
-__global__ void k_advance_step(TokIO* io) { io->t += 1; }
+
+// Called by every thread of every CTA at the very end of the launch that closes a
+// token: each CTA has read io->t at its start; the last CTA to get here (every other
+// one has counted itself, so every read is done) moves the record to the next token.
+__device__ __forceinline__ void tok_advance_if_last(TokIO* io) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+        if (atomicAdd(&io->done, 1u) == total - 1) {
+            io->done = 0;
+            io->t += 1;
+            __threadfence();
+        }
+    }
+}
 
 // ----------------------------------------------------------------- tile addressing
 // A "tile" is one gray block for one (layer, chain), or one stand-alone tau item.
 struct TileArgs {
-    // stack addressing
+    // stack addressing: layer l1's block reads act[l1][g] and adds onto act_out[l1][g]
+    // (for the tanh stack act_out = act + G L: layer l's output buffer is layer l+1's input)
     float* act;
+    float* act_out;
     const float* h;
     long long L;
     long long G;
@@ -126,7 +144,8 @@ struct TileArgs {
     long long spec_stride;  // complex entries per item
     const float2* tw;    // e^{-2 pi i k / 2^twlog}, k < 2^twlog
     int twlog;
-    const TokIO* io;     // non-null: n = io->t + 1 (replayed per-token graph), overwrite = n a power of 2
+    TokIO* io;           // non-null: n = io->t + 1 (replayed per-token graph), overwrite = n a power of 2
+    int advance;         // with io: this launch closes the token and advances the record
 };
 
 // The block position of a launch: from the arguments, or from the step record.
@@ -157,7 +176,7 @@ __device__ __forceinline__ TilePtrs tile_ptrs(const TileArgs& a, long long item)
         long long g = item - l1 * a.G;
         long long c = g % a.D;
         p.in = a.act + (l1 * a.G + g) * a.L + (a.n - a.U);
-        p.out = a.act + ((l1 + 1) * a.G + g) * a.L + a.n;
+        p.out = a.act_out + (l1 * a.G + g) * a.L + a.n;
         p.taps = a.h + (l1 * a.D + c) * a.L;
         p.spec = a.spec ? a.spec + (l1 * a.D + c) * a.spec_stride : nullptr;
     }
@@ -199,6 +218,7 @@ __global__ void __launch_bounds__(NT) k_tile_direct(TileArgs a0) {
             if (r < U) p.out[r] = a.overwrite ? acc[q] : p.out[r] + acc[q];
         }
     }
+    if (a.io && a.advance) tok_advance_if_last(a.io);
 }
 
 // ----------------------------------------------------------------- shared-memory FFT
@@ -490,6 +510,7 @@ __global__ void __launch_bounds__(FftTile<LOGN>::NT, FftTile<LOGN>::MINB) k_bloc
             fft_last_pass_store<LOGN, RB, 1, TWLOG>(X, t, T, a.tw, p.out, Os, a.overwrite, valid);
         }
     }
+    if (a.io && a.advance) tok_advance_if_last(a.io);
 }
 
 // ----------------------------------------------------------------- filter spectra
@@ -535,7 +556,8 @@ struct StepArgs {
     float* y;        // [G] y^M_t
     int closed;      // write a^M_t as token t+1
     int fuseU;       // edge of the block n = t+1 done here (0: none)
-    const TokIO* io; // non-null: t, x and y come from the step record (replayed graph)
+    TokIO* io;       // non-null: t, x and y come from the step record (replayed graph)
+    int advance;     // with io: this launch closes the token and advances the record
 };
 
 template <int NT>
@@ -558,39 +580,56 @@ __global__ void __launch_bounds__(NT) k_token_step(StepArgs a) {
             float av = xt ? xt[g] : a.act[g * a.L + t];
             a.act[g * a.L + t] = av;
             float y = 0.f;
-            for (int l = 1; l <= a.M; ++l) {
-                float* slot = a.act + ((long long)l * a.G + g) * a.L + t;
-                const float h0 = a.h[((long long)(l - 1) * a.D + c) * a.L];
-                const float p = (t == 0) ? 0.f : *slot;
-                y = fmaf(h0, av, p);
-                av = act_tanh(y);
-                *slot = av;
+            // the running sums and taps h_0 of the layers do not depend on the chain:
+            // eight layers' worth is loaded before their links run, so the chain waits for
+            // global memory once per eight layers, not once per layer
+            constexpr int KB = 8;
+            for (int l0 = 1; l0 <= a.M; l0 += KB) {
+                float pv[KB], hv[KB];
+#pragma unroll
+                for (int k = 0; k < KB; ++k) {
+                    const int l = l0 + k;
+                    const bool ok = l <= a.M;
+                    pv[k] = (ok && t > 0) ? a.act[((long long)l * a.G + g) * a.L + t] : 0.f;
+                    hv[k] = ok ? a.h[((long long)(l - 1) * a.D + c) * a.L] : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < KB; ++k) {
+                    const int l = l0 + k;
+                    if (l <= a.M) {
+                        y = fmaf(hv[k], av, pv[k]);
+                        av = act_tanh(y);
+                        a.act[((long long)l * a.G + g) * a.L + t] = av;
+                    }
+                }
             }
             yt[g] = y;
             if (a.closed && t + 1 < a.L) a.act[g * a.L + t + 1] = av;
         }
     }
     const int U = a.fuseU;
-    if (U == 0) return;
-    __syncthreads();
-    const long long n = t + 1;
-    const bool ow = is_pow2(n);
-    const int nch = (int)min(32LL, a.G - g0);
-    const int items = nch * a.M * U;
-    for (int it = threadIdx.x; it < items; it += NT) {
-        const int r = it % U;
-        const int rest = it / U;
-        const int i = rest % nch;
-        const int l = rest / nch + 1;
-        const long long g = g0 + i;
-        const long long c = g % a.D;
-        const float* in = a.act + ((long long)(l - 1) * a.G + g) * a.L + (n - U);
-        const float* hp = a.h + ((long long)(l - 1) * a.D + c) * a.L + U + r;
-        float acc = 0.f;
-        for (int j = 0; j < U; ++j) acc = fmaf(in[j], hp[-j], acc);
-        float* o = a.act + ((long long)l * a.G + g) * a.L + n + r;
-        *o = ow ? acc : *o + acc;
+    if (U != 0) {
+        __syncthreads();
+        const long long n = t + 1;
+        const bool ow = is_pow2(n);
+        const int nch = (int)min(32LL, a.G - g0);
+        const int items = nch * a.M * U;
+        for (int it = threadIdx.x; it < items; it += NT) {
+            const int r = it % U;
+            const int rest = it / U;
+            const int i = rest % nch;
+            const int l = rest / nch + 1;
+            const long long g = g0 + i;
+            const long long c = g % a.D;
+            const float* in = a.act + ((long long)(l - 1) * a.G + g) * a.L + (n - U);
+            const float* hp = a.h + ((long long)(l - 1) * a.D + c) * a.L + U + r;
+            float acc = 0.f;
+            for (int j = 0; j < U; ++j) acc = fmaf(in[j], hp[-j], acc);
+            float* o = a.act + ((long long)l * a.G + g) * a.L + n + r;
+            *o = ow ? acc : *o + acc;
+        }
     }
+    if (a.io && a.advance) tok_advance_if_last(a.io);
 }
 
 // ----------------------------------------------------------------- window kernel

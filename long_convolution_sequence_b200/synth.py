@@ -129,6 +129,39 @@ def start_token(B: int, D: int, seed: int = 0) -> np.ndarray:
     return _rng(seed, 3).standard_normal((B, D)).astype(np.float32)
 
 
+def _bf16_values(a: np.ndarray) -> np.ndarray:
+    """float32 array holding the nearest bfloat16 values (torch's conversion): the GEMM
+    weights of the Hyena-like model are bf16 tensors."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def hyena_params(M: int, D: int, L: int, V: int, seed: int = 0) -> dict:
+    """Random-init weights of the Hyena-like model (stream 4, one sub-stream per layer):
+    embedding E [V][D] ~ N(0, 1); per layer W_in [3D][D] ~ N(0, 1/D), short-conv taps
+    c [3][3D] ~ N(0, 1/3), W1 [4D][D] ~ N(0, 1/D), W2 [D][4D] ~ N(0, 1/(4D)); LM head
+    W_lm [V][D] ~ N(0, 1/D); the GEMM weights (E, W_in, W1, W2, W_lm) rounded to bf16
+    values.  The long-convolution filters h [M][D][L] follow the mixer's law
+    (``filters``, same seed)."""
+    g = _rng(seed, 4, 0)
+    E = _bf16_values(g.standard_normal((V, D)))
+    W_lm = _bf16_values(g.standard_normal((V, D)) / math.sqrt(D))
+    W_in, c, W1, W2 = [], [], [], []
+    for l in range(M):
+        gl = _rng(seed, 4, 1 + l)
+        W_in.append(_bf16_values(gl.standard_normal((3 * D, D)) / math.sqrt(D)))
+        c.append((gl.standard_normal((3, 3 * D)) / math.sqrt(3.0)).astype(np.float32))
+        W1.append(_bf16_values(gl.standard_normal((4 * D, D)) / math.sqrt(D)))
+        W2.append(_bf16_values(gl.standard_normal((D, 4 * D)) / math.sqrt(4 * D)))
+    h = filters(M, D, L, seed=seed)
+    return {"E": E, "W_lm": W_lm, "W_in": W_in, "c": c, "W1": W1, "W2": W2, "h": list(h)}
+
+
+def token_ids(T: int, B: int, V: int, seed: int = 0) -> np.ndarray:
+    """int32 [T][B] synthetic token ids, uniform over the vocabulary (stream 5)."""
+    return _rng(seed, 5).integers(0, V, size=(T, B)).astype(np.int32)
+
+
 # Workloads (layers, B, D, L) of the measured configurations.
 CONFIGS = {
     "tiny": dict(M=1, B=1, D=16, L=1 << 10),

@@ -1,4 +1,5 @@
-"""The Lazy and Eager baselines (FI_PATH_LAZY / FI_PATH_EAGER) against the oracle.
+"""The Lazy and Eager baselines (FI_PATH_LAZY / FI_PATH_EAGER, and their non-parallel
+forms FI_PATH_LAZY_NP / FI_PATH_EAGER_NP) against the oracle.
 
 Both evaluate the same stack as the relaxed tiling by the two plain strategies of the
 Flash Inference summary's section "Kern-Algorithmus: Relaxierte
@@ -18,7 +19,8 @@ from long_convolution_sequence_b200 import synth
 TOL_TF = 1e-4   # teacher-forced: max |err| / RMS(y)
 TOL_CL = 1e-3   # closed loop
 
-PATHS = {"lazy": fi.FI_PATH_LAZY, "eager": fi.FI_PATH_EAGER}
+PATHS = {"lazy": fi.FI_PATH_LAZY, "eager": fi.FI_PATH_EAGER,
+         "lazy_np": fi.FI_PATH_LAZY_NP, "eager_np": fi.FI_PATH_EAGER_NP}
 
 
 def rel(got, ref):

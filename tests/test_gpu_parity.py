@@ -274,9 +274,10 @@ def test_token_path_graphs_replay_the_eager_launches(closed):
                 ctx.forward(x[:700], 700, y[:700])
                 ctx.forward(x[700:], L - 700, y[700:])
             if graphs:
-                # per token: step kernel, block launch unless fused into it, advance;
-                # per call one record write
-                assert L * 2 + 2 <= ctx.info().launches - n0 <= L * 3 + 2
+                # per token: the step kernel and the block launch unless the block is fused
+                # into the step kernel (or the last token, which releases none); per call
+                # one record write
+                assert L + 2 <= ctx.info().launches - n0 <= L * 2 + 2
             outs.append(y)
     np.testing.assert_array_equal(outs[0], outs[1])
     np.testing.assert_array_equal(outs[0], outs[2])
@@ -305,6 +306,35 @@ def test_step_calls_with_changing_pointers_replay_graphs():
             got[t] = yh[t]
         assert ctx.info().t == L
     assert rel(got, ref) < TOL_TF
+
+
+@pytest.mark.parametrize("path", ["window", "token"])
+def test_traced_runs_report_every_launch(path):
+    # tracing brackets every launch with events, on the captured window path and on the
+    # host-issued per-token path; the per-launch list covers the whole run, in order
+    M, B, D, L = 3, 1, 8, 1024
+    h = synth.filters(M, D, L, seed=10)
+    x0 = synth.start_token(B, D, seed=10)
+    ref = oracle.stack(h, x0, T=L, closed_loop=True, want=("y_last",))["y_last"]
+    with fi.FlashInference(M, B, D, L, h) as ctx:
+        ctx.set_path(fi.FI_PATH_WINDOW if path == "window" else fi.FI_PATH_TOKEN)
+        ctx.set_trace(True)
+        out = np.empty((L, B, D), np.float32)
+        n0 = ctx.info().launches
+        ctx.generate(x0, L, out)
+        n = ctx.info().launches - n0
+        cls, q, us = ctx.trace_launches()
+        assert len(cls) == n and (us > 0).all()
+        if path == "token":
+            assert (cls == fi.FI_K_TOKEN_STEP).sum() == L
+        else:
+            W = ctx.info().window
+            assert (cls == fi.FI_K_WINDOW).sum() == L // W
+            assert sorted(q[cls != fi.FI_K_WINDOW].tolist()) == sorted((k & -k).bit_length() - 1
+                                                                    for k in range(W, L, W))
+        per_class = ctx.trace()
+        assert sum(v[0] for v in per_class.values()) == n
+    assert rel(out, ref) < TOL_CL
 
 
 @pytest.mark.parametrize("force", ["direct", "fft"])
