@@ -158,9 +158,10 @@ int fi_forward(fi_ctx *ctx, const float *x, int steps, float *y);
  * so fi_generate / fi_forward / fi_step continue the sequence.  Needs t = 0 (after
  * fi_create or fi_reset) and a tiled path (FI_PATH_WINDOW or FI_PATH_TOKEN), else
  * FI_EINVAL; 1 <= p <= L.  Prompts shorter than 8 tokens take the online path.
- * The context keeps about 4 * B * D * (4U + M U / 2) bytes of device scratch from the
- * first prefill of that size on (FI_ENOMEM if it cannot get it), freed with the
- * context.  Asynchronous on the context's stream like fi_forward; with host buffers
+ * The context keeps 4 * B * D * (2U + M (p - n0)) bytes of device scratch (n0 the
+ * largest power of two <= p) and the spectra of the shifted taps of the prompt's size,
+ * 8 * M * D * (U + 2) bytes, made by the first prefill of that size and reused by later
+ * ones (FI_ENOMEM if it cannot get them); both are freed with the context.  Asynchronous on the context's stream like fi_forward; with host buffers
  * it synchronises before returning. */
 int fi_prefill(fi_ctx *ctx, const float *x, int p, float *y);
 
@@ -293,6 +294,11 @@ int fi_lm_forward(fi_lm *m, const int *tokens, int steps, float *logits, int *ne
  * (NULL: continue from the previous call's last choice; required at t = 0); next
  * [steps][B] receives each step's choice, which is the following step's input. */
 int fi_lm_generate(fi_lm *m, const int *tok0, int steps, int *next);
+
+/* Greedy generation replays one captured CUDA graph per block size ([Impl]: the
+ * launches of one token recorded once; the token index read from device memory) when
+ * on (the default); off, or with tracing on, every launch is issued from the host. */
+int fi_lm_set_graphs(fi_lm *m, int on);
 
 /* Tracing (off by default): later calls record events around every block launch of
  * the mixers and around the mixer steps of every 64th token. */

@@ -71,6 +71,7 @@ SIGNATURES = {
     "fi_lm_forward": (_I, [_P, _P, _I, _P, _P]),
     "fi_lm_generate": (_I, [_P, _P, _I, _P]),
     "fi_lm_set_trace": (_I, [_P, _I]),
+    "fi_lm_set_graphs": (_I, [_P, _I]),
     "fi_lm_split": (_I, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     "fi_last_error": (ctypes.c_char_p, []),
     "fi_version": (ctypes.c_char_p, []),
@@ -274,6 +275,9 @@ class LanguageModel:
 
     def set_trace(self, on: bool):
         _check(get_lib().fi_lm_set_trace(self._h, int(bool(on))))
+
+    def set_graphs(self, on: bool):
+        _check(get_lib().fi_lm_set_graphs(self._h, int(bool(on))))
 
     def split(self):
         """(mixer_us, total_us) of the last traced call."""

@@ -120,6 +120,9 @@ struct fi_ctx {
     size_t sy_n = 0;
     float* pre = nullptr;  // prompt-prefill scratch, grown on demand
     size_t pre_n = 0;
+    float2* pre_spec = nullptr;  // prefill: spectra of the shifted taps [M][D][U+2] of one prompt size
+    int pre_spec_q = -1;         // its block size 2^q (-1: none)
+    size_t pre_spec_n = 0;
     std::map<GraphKey, GraphEntry> gcache;
     std::vector<GraphKey> gorder;
     // per-token path: one graph per (mode, block size 2^q released after the token;
@@ -426,7 +429,7 @@ bool win_fixed_geom(const fi_ctx* c, int W) {
 }
 
 template <int W, int MAXM>
-int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
+int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st, int pdl) {
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)c->win_ncta);
@@ -434,7 +437,7 @@ int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
     cfg.dynamicSmemBytes = c->win_smem;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
-    set_pdl(&cfg, at, c->pdl);
+    set_pdl(&cfg, at, pdl);
     if constexpr (W == 128 && MAXM == 18) {
         if (win_fixed_geom(c, W)) {
             CK(cudaLaunchKernelEx(&cfg, k_window<W, MAXM, true, kWinCPBT>, a));
@@ -446,22 +449,22 @@ int launch_window_t(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
 }
 
 template <int W>
-int launch_window_w(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
+int launch_window_w(const fi_ctx* c, const WinArgs& a, cudaStream_t st, int pdl) {
     switch (win_maxm(c->M)) {
-        case 8: return launch_window_t<W, 8>(c, a, st);
-        case 18: return launch_window_t<W, 18>(c, a, st);
-        case 20: return launch_window_t<W, 20>(c, a, st);
-        case 40: return launch_window_t<W, 40>(c, a, st);
+        case 8: return launch_window_t<W, 8>(c, a, st, pdl);
+        case 18: return launch_window_t<W, 18>(c, a, st, pdl);
+        case 20: return launch_window_t<W, 20>(c, a, st, pdl);
+        case 40: return launch_window_t<W, 40>(c, a, st, pdl);
         default: return set_err(FI_EINVAL, "window kernel supports at most 40 layers");
     }
 }
 
-int launch_window(const fi_ctx* c, const WinArgs& a, cudaStream_t st) {
+int launch_window(const fi_ctx* c, const WinArgs& a, cudaStream_t st, int pdl) {
     switch (c->W) {
-        case 32: return launch_window_w<32>(c, a, st);
-        case 64: return launch_window_w<64>(c, a, st);
-        case 128: return launch_window_w<128>(c, a, st);
-        case 256: return launch_window_w<256>(c, a, st);
+        case 32: return launch_window_w<32>(c, a, st, pdl);
+        case 64: return launch_window_w<64>(c, a, st, pdl);
+        case 128: return launch_window_w<128>(c, a, st, pdl);
+        case 256: return launch_window_w<256>(c, a, st, pdl);
         default: return set_err(FI_EINVAL, "unsupported window %d", c->W);
     }
 }
@@ -810,6 +813,7 @@ int run_token_graphs(fi_ctx* c, long long t0, long long steps, const float* x, f
         }
     }
     TokIO v;
+    memset(&v, 0, sizeof(v));
     v.x = x;
     v.y = out;
     v.tx = t0;
@@ -856,7 +860,9 @@ int enqueue_window_path(fi_ctx* c, long long t0, long long steps, const float* x
         int rc;
         {
             LaunchScope scope(c, FI_K_WINDOW, st);
-            rc = launch_window(c, a, st);
+            // the call's first launch follows the staging copies of its inputs, which
+            // griddepcontrol.wait does not wait for: no programmatic dependent launch
+            rc = launch_window(c, a, st, t == t0 ? 0 : c->pdl);
         }
         if (rc) return rc;
         if (t1 == (k + 1) * W && t1 < L) {
@@ -1109,6 +1115,7 @@ void free_ctx(fi_ctx* c) {
     cudaFree(c->sx);
     cudaFree(c->sy);
     cudaFree(c->pre);
+    cudaFree(c->pre_spec);
     cudaFree(c->tio);
     for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
     if (c->cap) cudaStreamDestroy(c->cap);
@@ -1169,41 +1176,64 @@ int prefill_impl(fi_ctx* c, const float* x, int p, float* y) {
     cudaStream_t st = c->stream;
     long long n0 = 1;
     while (2 * n0 <= p) n0 <<= 1;  // the first open block: the largest power of two <= p
-    // scratch (kept by the context): blocks [G][U], out [G][U], taps [G][2U], spectra
-    // [G][U + 2] complex, the saved activations [M][G][p - n0]
-    const size_t nb = (size_t)G * U, nspec = (size_t)G * fused_stride(U);
-    const size_t need = 4 * nb + 2 * nspec + (size_t)M * G * (size_t)(p - n0);
+    // scratch (kept by the context): blocks [G][U], out [G][U] (together the shifted taps
+    // [D][2U] while the spectra are made), the saved activations [M][G][p - n0]
+    const size_t nb = (size_t)G * U;
+    const size_t need = 2 * nb + (size_t)M * G * (size_t)(p - n0);
     int rc;
     if ((rc = ensure_stage(c, &c->pre, &c->pre_n, need))) return rc;
     float* blocks = c->pre;
     float* out = blocks + nb;
-    float* taps = out + nb;
-    float2* spec = reinterpret_cast<float2*>(taps + 2 * nb);  // 8-byte aligned: 4 nb floats before it
-    float* saved_area = reinterpret_cast<float*>(spec + nspec);
+    float* saved_area = out + nb;
     const int grid = 4 * c->nsm, nt = 256;
+    const long long sstride = fused_stride(U);
+    // the spectra of the shifted taps of every layer and channel, once per prompt size
+    // (the FFT precompute of section "Speicheroptimierung" for the prompt's block size);
+    // the batch rows of a channel share them
+    if (c->pre_spec_q != q) {
+        const size_t ns = (size_t)M * c->D * sstride;
+        if (c->pre_spec_n < ns) {
+            CK(cudaStreamSynchronize(st));
+            cudaFree(c->pre_spec);
+            c->bytes -= c->pre_spec_n * sizeof(float2);
+            c->pre_spec = nullptr;
+            c->pre_spec_n = 0;
+            c->pre_spec_q = -1;
+            if ((rc = dev_alloc(c, &c->pre_spec, ns))) return rc;
+            c->pre_spec_n = ns;
+        }
+        float* taps = blocks;  // [D][2U]: within blocks and out, 2 G U >= 2 D U floats
+        for (int l = 1; l <= M; ++l) {
+            k_prefill_taps<<<grid, nt, 0, st>>>(c->h, l, c->D, c->D, L, U, taps);
+            if ((rc = make_spectra(q, taps, 2 * U, c->D, c->pre_spec + (size_t)(l - 1) * c->D * sstride, c->tw,
+                                   st)))
+                return rc;
+        }
+        CK(cudaGetLastError());
+        c->pre_spec_q = q;
+    }
     k_prefill_input<<<grid, nt, 0, st>>>(x, G, L, p, c->act);
     long long nl = 1;
     for (int l = 1; l <= M; ++l) {
         k_prefill_gather<<<grid, nt, 0, st>>>(c->act, l - 1, G, L, p, U, blocks);
-        k_prefill_taps<<<grid, nt, 0, st>>>(c->h, l, c->D, G, L, U, taps);
-        if ((rc = make_spectra(q, taps, 2 * U, (int)G, spec, c->tw, st))) return rc;
         TileArgs a;
         memset(&a, 0, sizeof(a));
         a.flat = 1;
         a.fin = blocks;
         a.fout = out;
-        a.ftaps = taps;
+        a.ftaps = blocks;  // not read: the FFT tau reads only the spectra
         a.ldt = 2 * U;
         a.U = U;
         a.count = (int)G;
         a.overwrite = 1;
         a.tw = c->tw;
         a.twlog = kTwLog;
-        a.spec = spec;
-        a.spec_stride = fused_stride(U);
+        a.spec = c->pre_spec + (size_t)(l - 1) * c->D * sstride;
+        a.spec_stride = sstride;
+        a.spec_mod = c->D;  // chain g = b D + c reads channel c's row
         if ((rc = launch_fft(q, a, st))) return rc;
         k_prefill_scatter<<<grid, nt, 0, st>>>(out, l, G, L, p, U, c->act, l == M ? y : nullptr);
-        nl += 5;
+        nl += 3;
     }
     CK(cudaGetLastError());
     float* saved = nullptr;
@@ -1256,6 +1286,9 @@ struct fi_lm {
     std::vector<std::pair<int, int>> ev_blocks, ev_steps;  // event index pairs
     int ev_call0 = -1, ev_call1 = -1;
     long long traced_tokens = 0, sampled_tokens = 0;
+    // greedy generation from captured graphs: one per block size released (32: none)
+    int graphs = 1;
+    cudaGraphExec_t gen_graph[33] = {};
 };
 
 namespace {
@@ -1312,48 +1345,116 @@ void lm_clear_trace(fi_lm* m) {
     m->traced_tokens = m->sampled_tokens = 0;
 }
 
+// Launch with programmatic dependent launch (the model's kernels wait for their
+// predecessors themselves, after prefetching what does not depend on them).
+template <typename... KArgs, typename... Args>
+int lm_launch(int pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+              Args... args) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    set_pdl(&cfg, at, pdl);
+    CK(cudaLaunchKernelEx(&cfg, kernel, args...));
+    return FI_OK;
+}
+
 template <int EPI>
-int lm_gemv(const __nv_bfloat16* W, int N, int K, const float* x, int B, int ln, float* y, cudaStream_t st) {
+int lm_gemv(int pdl, const __nv_bfloat16* W, int N, int K, const float* x, int B, int ln, float* y,
+            cudaStream_t st) {
     const int rows_per_cta = kLmThreads / 32;
     const int grid = std::min((N + rows_per_cta - 1) / rows_per_cta, 8 * 148);
-    k_lm_gemv<EPI><<<grid, kLmThreads, (size_t)B * K * sizeof(float), st>>>(W, N, K, x, B, ln, y);
-    CK(cudaGetLastError());
-    return FI_OK;
+    return lm_launch(pdl, k_lm_gemv<EPI>, dim3(grid), dim3(kLmThreads), (size_t)B * K * sizeof(float), st, W, N, K, x,
+                     B, ln, y);
 }
 
 // One token t: tok_src [B] (device) is its input; logits_out [B][V] (device) or null;
 // next_out [B] (device) receives the greedy choice, also kept as the next input.
-int lm_token(fi_lm* m, long long t, const int* tok_src, float* logits_out, int* next_out, cudaStream_t st) {
+// first: the token's first launch follows copies or a memset of the call's set-up, which
+// griddepcontrol.wait does not wait for, so it is launched without programmatic
+// dependent launch; tracing also turns it off (overlapping launches blur the events).
+int lm_token(fi_lm* m, long long t, const int* tok_src, float* logits_out, int* next_out, cudaStream_t st,
+             TokIO* io = nullptr, bool first = false) {
     const int M = m->M, B = m->B, D = m->D, V = m->V;
     const long long L = m->L, G = (long long)B * D;
     fi_ctx* c = m->mix;
+    // Programmatic dependent launch is left off here: with every kernel releasing its
+    // successor at once, launches cascade and the waiting CTAs of later kernels crowd
+    // the running one (measured on the 18-layer model: 35.7 s per 32768-token generation
+    // with it, 27.5 s without).
+    const int pdl = 0;
+    (void)first;
     int rc;
-    k_lm_embed<<<(B * D + 255) / 256, 256, 0, st>>>(m->E, tok_src, B, D, m->u);
+    if ((rc = lm_launch(first ? 0 : pdl, k_lm_embed, dim3((B * D + 255) / 256), dim3(256), 0, st, (const __nv_bfloat16*)m->E,
+                        tok_src, B, D, m->u)))
+        return rc;
     const bool sample = m->trace_on && (t % kTraceEvery == 0);
     for (int l = 0; l < M; ++l) {
-        if ((rc = lm_gemv<kLmStore>(m->Win + (size_t)l * 3 * D * D, 3 * D, D, m->u, B, 1, m->z, st))) return rc;
+        if ((rc = lm_gemv<kLmStore>(pdl, m->Win + (size_t)l * 3 * D * D, 3 * D, D, m->u, B, 1, m->z, st))) return rc;
         const int e0 = sample ? lm_event(m, st) : -1;
-        k_lm_mixer<<<(B * D + 127) / 128, 128, 0, st>>>(m->z, m->zr + (size_t)l * 2 * B * 3 * D,
-                                                       m->conv + (size_t)l * 9 * D, c->h + (size_t)l * D * L, L, B,
-                                                       D, t, c->act + (size_t)l * G * L, c->yout + (size_t)l * G * L,
-                                                       m->u);
+        if ((rc = lm_launch(pdl, k_lm_mixer, dim3((B * D + 127) / 128), dim3(128), 0, st, (const float*)m->z,
+                            m->zr + (size_t)l * 2 * B * 3 * D, (const float*)(m->conv + (size_t)l * 9 * D),
+                            (const float*)(c->h + (size_t)l * D * L), L, B, D, t, c->act + (size_t)l * G * L,
+                            c->yout + (size_t)l * G * L, m->u, (const TokIO*)io)))
+            return rc;
         if (sample) m->ev_steps.push_back({e0, lm_event(m, st)});
-        CK(cudaGetLastError());
-        if ((rc = lm_gemv<kLmGelu>(m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->u, B, 1, m->m1, st))) return rc;
-        if ((rc = lm_gemv<kLmAdd>(m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, st))) return rc;
+        if ((rc = lm_gemv<kLmGelu>(pdl, m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->u, B, 1, m->m1, st))) return rc;
+        if ((rc = lm_gemv<kLmAdd>(pdl, m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, st))) return rc;
     }
     float* lg = logits_out ? logits_out : m->logits;
-    if ((rc = lm_gemv<kLmStore>(m->Wlm, V, D, m->u, B, 1, lg, st))) return rc;
-    k_lm_argmax<<<B, 256, 0, st>>>(lg, V, m->tok, next_out);
-    CK(cudaGetLastError());
-    if (t + 1 < L) {
+    if ((rc = lm_gemv<kLmStore>(pdl, m->Wlm, V, D, m->u, B, 1, lg, st))) return rc;
+    const bool block_follows = t + 1 < L;
+    if ((rc = lm_launch(pdl, k_lm_argmax, dim3(B), dim3(256), 0, st, (const float*)lg, V, m->tok, next_out, io,
+                        (io && !block_follows) ? 1 : 0)))
+        return rc;
+    if (block_follows) {
         const int e0 = m->trace_on ? lm_event(m, st) : -1;
-        if ((rc = launch_block(c, t + 1, tau_of(c, ctz64(t + 1)), st))) return rc;
+        if ((rc = launch_block(c, t + 1, tau_of(c, ctz64(t + 1)), st, 0, 0, io))) return rc;  // the block kernels read through L1: no early start
         if (m->trace_on) m->ev_blocks.push_back({e0, lm_event(m, st)});
     }
     if (m->trace_on) {
         m->traced_tokens++;
         if (sample) m->sampled_tokens++;
+    }
+    return FI_OK;
+}
+
+int lm_run_graphs(fi_lm* m, int steps, int* next_d, cudaStream_t st) {
+    fi_ctx* c = m->mix;
+    const long long t0 = m->t;
+    for (long long t = t0; t < t0 + steps; ++t) {  // capture what this call needs first
+        const int idx = t + 1 < m->L ? ctz64(t + 1) : 32;
+        if (m->gen_graph[idx]) continue;
+        const long long tr = idx == 32 ? m->L - 1 : (1LL << idx) - 1;  // a token releasing 2^idx
+        CK(cudaStreamBeginCapture(c->cap, cudaStreamCaptureModeRelaxed));
+        int rc = lm_token(m, tr, m->tok, nullptr, nullptr, c->cap, c->tio, true);
+        cudaGraph_t graph = nullptr;
+        cudaError_t e = cudaStreamEndCapture(c->cap, &graph);
+        if (rc || e != cudaSuccess) {
+            if (graph) cudaGraphDestroy(graph);
+            cudaGetLastError();
+            return rc ? rc : set_err(FI_ECUDA, "model graph capture failed: %s", cudaGetErrorString(e));
+        }
+        e = cudaGraphInstantiate(&m->gen_graph[idx], graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) {
+            m->gen_graph[idx] = nullptr;
+            return set_err(FI_ECUDA, "model graph instantiate failed: %s", cudaGetErrorString(e));
+        }
+    }
+    TokIO v;
+    memset(&v, 0, sizeof(v));
+    v.tx = t0;
+    v.t = t0;
+    v.itok = next_d;
+    k_set_step<<<1, 1, 0, st>>>(c->tio, v);
+    CK(cudaGetLastError());
+    for (long long t = t0; t < t0 + steps; ++t) {
+        const int idx = t + 1 < m->L ? ctz64(t + 1) : 32;
+        CK(cudaGraphLaunch(m->gen_graph[idx], st));
     }
     return FI_OK;
 }
@@ -1416,11 +1517,16 @@ int lm_run(fi_lm* m, const int* tokens, const int* tok0, int steps, float* logit
         lm_clear_trace(m);
         m->ev_call0 = lm_event(m, st);
     }
-    for (int k = 0; k < steps; ++k) {
-        const int* src = tokens ? tok_d + (size_t)k * B : m->tok;
-        if ((rc = lm_token(m, m->t + k, src, logits ? logits_d + (size_t)k * B * V : nullptr,
-                           next_d + (size_t)k * B, st)))
-            return rc;
+    if (!tokens && m->graphs && !m->trace_on) {
+        // greedy generation: one captured graph per block size, the token from the record
+        if ((rc = lm_run_graphs(m, steps, next_d, st))) return rc;
+    } else {
+        for (int k = 0; k < steps; ++k) {
+            const int* src = tokens ? tok_d + (size_t)k * B : m->tok;
+            if ((rc = lm_token(m, m->t + k, src, logits ? logits_d + (size_t)k * B * V : nullptr,
+                               next_d + (size_t)k * B, st, nullptr, k == 0)))
+                return rc;
+        }
     }
     if (m->trace_on) m->ev_call1 = lm_event(m, st);
     m->t += steps;
@@ -1433,6 +1539,8 @@ int lm_run(fi_lm* m, const int* tokens, const int* tok0, int steps, float* logit
 void lm_free(fi_lm* m) {
     if (!m) return;
     lm_clear_trace(m);
+    for (int i = 0; i < 33; ++i)
+        if (m->gen_graph[i]) cudaGraphExecDestroy(m->gen_graph[i]);
     if (m->mix) {
         cudaStreamSynchronize(m->mix->stream);
         cudaFree(m->mix->yout);
@@ -1897,6 +2005,13 @@ int fi_lm_generate(fi_lm* m, const int* tok0, int steps, int* next) {
     int rc = check_lm(m);
     if (rc) return rc;
     return lm_run(m, nullptr, tok0, steps, nullptr, next);
+}
+
+int fi_lm_set_graphs(fi_lm* m, int on) {
+    int rc = check_lm(m);
+    if (rc) return rc;
+    m->graphs = on ? 1 : 0;
+    return FI_OK;
 }
 
 int fi_lm_set_trace(fi_lm* m, int on) {

@@ -98,6 +98,7 @@ struct TokIO {
     long long t;     // token being processed
     int closed;
     unsigned done;   // CTAs of the current launch that have finished (advancing launch only)
+    int* itok;       // language model: greedy choices [.][B] from token tx on
 };
 
 __global__ void k_set_step(TokIO* io, TokIO v) { *io = v; }
@@ -142,6 +143,7 @@ struct TileArgs {
     int overwrite;   // 1: store, 0: accumulate
     const float2* spec;  // spectra of this block size (FFT)
     long long spec_stride;  // complex entries per item
+    long long spec_mod;     // flat addressing: item i reads spectrum row i % spec_mod (0: row i)
     const float2* tw;    // e^{-2 pi i k / 2^twlog}, k < 2^twlog
     int twlog;
     TokIO* io;           // non-null: n = io->t + 1 (replayed per-token graph), overwrite = n a power of 2
@@ -170,7 +172,7 @@ __device__ __forceinline__ TilePtrs tile_ptrs(const TileArgs& a, long long item)
         p.in = a.fin + item * a.U;
         p.out = a.fout + item * a.U;
         p.taps = a.ftaps + item * a.ldt;
-        p.spec = a.spec ? a.spec + item * a.spec_stride : nullptr;
+        p.spec = a.spec ? a.spec + (a.spec_mod ? item % a.spec_mod : item) * a.spec_stride : nullptr;
     } else {
         long long l1 = item / a.G;  // layer - 1
         long long g = item - l1 * a.G;

@@ -102,3 +102,21 @@ def test_trace_reports_a_mixer_share():
         lm.generate(np.array([1, 2], np.int32), L, nxt)
         mix, tot = lm.split()
         assert 0 < mix < tot
+
+
+def test_generation_from_graphs_equals_host_launches():
+    # the replayed per-token graphs run the same kernels on the same data: identical choices
+    M, B, D, L, V = 2, 3, 32, 256, 300
+    p = synth.hyena_params(M, D, L, V, seed=11)
+    tok0 = np.array([5, 17, 200], np.int32)
+    outs = []
+    with model(p, M, B, D, L, V) as lm:
+        for graphs in (True, False, True):
+            lm.reset()
+            lm.set_graphs(graphs)
+            nxt = np.empty((L, B), np.int32)
+            lm.generate(tok0, 100, nxt[:100])      # two calls: the record is set again
+            lm.generate(None, L - 100, nxt[100:])
+            outs.append(nxt)
+    np.testing.assert_array_equal(outs[0], outs[1])
+    np.testing.assert_array_equal(outs[0], outs[2])
