@@ -271,13 +271,20 @@ __global__ void __launch_bounds__(ClusterTile<LOGNC, LOGN2>::T, ClusterTile<LOGN
 #pragma unroll
             for (int u = 0; u < NPT; ++u) g[u][c] = Xc[fft::pad(k1 * PER + t + u * T)];
         }
-        // this CTA's reads of the others' shared memory are done (release); the wait,
-        // before exit, overlaps the output stores
-        asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+
+        float dep = 0.f;
+#pragma unroll
+        for (int u = 0; u < NPT; ++u) {
+            fft::dft<NC>(g[u]);
+            dep += g[u][0].x;  // every DFT output depends on every value loaded for it
+        }
+        // every value read from the other CTAs' shared memory has arrived (the arrival
+        // takes an operand computed from all of them), so this CTA no longer reads them
+        // and a relaxed arrival suffices; the wait, before exit, overlaps the stores
+        asm volatile("barrier.cluster.arrive.relaxed.aligned; // %0\n" ::"f"(dep) : "memory");
 #pragma unroll
         for (int u = 0; u < NPT; ++u) {
             const int j = t + u * T;
-            fft::dft<NC>(g[u]);
 #pragma unroll
             for (int n1 = NC / 2; n1 < NC; ++n1) {
                 const float2 F = g[u][fft::omap<NC>(n1)];
