@@ -353,6 +353,17 @@ int launch_spectra_cluster(int q, const float* taps, long long ld, int count, fl
 }
 
 int launch_direct_tile(const TileArgs& a, cudaStream_t st) {
+    if (a.U <= 8 && (a.U & (a.U - 1)) == 0) {
+        const unsigned grid = (unsigned)((a.count + 127) / 128);
+        switch (a.U) {
+            case 1: k_tile_direct_small<1><<<grid, 128, 0, st>>>(a); break;
+            case 2: k_tile_direct_small<2><<<grid, 128, 0, st>>>(a); break;
+            case 4: k_tile_direct_small<4><<<grid, 128, 0, st>>>(a); break;
+            default: k_tile_direct_small<8><<<grid, 128, 0, st>>>(a); break;
+        }
+        CK(cudaGetLastError());
+        return FI_OK;
+    }
     const size_t smem = (size_t)3 * a.U * sizeof(float);
     k_tile_direct<kDirectNT, 4><<<a.count, kDirectNT, smem, st>>>(a);
     CK(cudaGetLastError());
@@ -1273,8 +1284,9 @@ struct fi_lm {
     long long t = 0;
     __nv_bfloat16 *E = nullptr, *Wlm = nullptr, *Win = nullptr, *W1 = nullptr, *W2 = nullptr;
     float* conv = nullptr;                       // [M][3][3D]
-    float *u = nullptr, *z = nullptr, *zr = nullptr, *m1 = nullptr, *logits = nullptr;
+    float *u = nullptr, *z = nullptr, *zr = nullptr, *m1 = nullptr;
     int *tok = nullptr, *next = nullptr;         // [B]: the next input token, the latest choice
+    unsigned long long* amax = nullptr;          // [B]: the LM head's running greedy choice (keys of lm_key)
     int* stage_i = nullptr;                      // host token arrays staged on the device
     size_t stage_i_n = 0;
     float* stage_f = nullptr;
@@ -1362,13 +1374,31 @@ int lm_launch(int pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return FI_OK;
 }
 
-template <int EPI>
-int lm_gemv(int pdl, const __nv_bfloat16* W, int N, int K, const float* x, int B, int ln, float* y,
-            cudaStream_t st) {
-    const int rows_per_cta = kLmThreads / 32;
-    const int grid = std::min((N + rows_per_cta - 1) / rows_per_cta, 8 * 148);
-    return lm_launch(pdl, k_lm_gemv<EPI>, dim3(grid), dim3(kLmThreads), (size_t)B * K * sizeof(float), st, W, N, K, x,
-                     B, ln, y);
+// Matrix-vector shapes: a warp per row slice of K / KS, RPW rows a warp at a time.
+// W_in and W1 (K = D) take two rows a warp, the LM head (K = D, N = V rows) four; W2
+// (K = 4D) splits each row over 4 warps, two rows a warp, so that either way a lane has
+// all of its loads for a step in flight together and each shared-memory read of the
+// inputs serves two or four rows.  At most kLmCtasPerSm CTAs an SM (one wave).
+template <int EPI, int KS, int RPW>
+int lm_gemv(int pdl, int nsm, const __nv_bfloat16* W, int N, int K, const float* x, int B, int ln, float* y,
+            unsigned long long* amax, cudaStream_t st) {
+    const int rows_per_cta = ((kLmThreads / 32) / KS) * RPW;
+    const int grid = std::min((N + rows_per_cta - 1) / rows_per_cta, kLmCtasPerSm * nsm);
+    const size_t smem = (size_t)B * K * sizeof(float);
+    if (B <= 4)
+        return lm_launch(pdl, k_lm_gemv<EPI, KS, RPW, 4>, dim3(grid), dim3(kLmThreads), smem, st, W, N, K, x, B, ln, y,
+                         amax);
+    return lm_launch(pdl, k_lm_gemv<EPI, KS, RPW, kLmMaxB>, dim3(grid), dim3(kLmThreads), smem, st, W, N, K, x, B, ln,
+                     y, amax);
+}
+
+template <int EPI, int KS, int RPW>
+int lm_gemv_attrs() {
+    CK(cudaFuncSetAttribute(k_lm_gemv<EPI, KS, RPW, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)kSmemMax - 1024));
+    CK(cudaFuncSetAttribute(k_lm_gemv<EPI, KS, RPW, kLmMaxB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)kSmemMax - 1024));
+    return FI_OK;
 }
 
 // One token t: tok_src [B] (device) is its input; logits_out [B][V] (device) or null;
@@ -1381,19 +1411,17 @@ int lm_token(fi_lm* m, long long t, const int* tok_src, float* logits_out, int* 
     const int M = m->M, B = m->B, D = m->D, V = m->V;
     const long long L = m->L, G = (long long)B * D;
     fi_ctx* c = m->mix;
-    // Programmatic dependent launch is left off here: with every kernel releasing its
-    // successor at once, launches cascade and the waiting CTAs of later kernels crowd
-    // the running one (measured on the 18-layer model: 35.7 s per 32768-token generation
-    // with it, 27.5 s without).
-    const int pdl = 0;
-    (void)first;
+    // Programmatic dependent launch: each kernel releases its successor once its own
+    // wait has returned, so at most one launch waits behind the running one (its weight
+    // rows already streaming into L2).  Tracing turns it off.
+    const int pdl = m->trace_on ? 0 : 1;
     int rc;
     if ((rc = lm_launch(first ? 0 : pdl, k_lm_embed, dim3((B * D + 255) / 256), dim3(256), 0, st, (const __nv_bfloat16*)m->E,
-                        tok_src, B, D, m->u)))
+                        tok_src, B, D, m->u, m->amax)))
         return rc;
     const bool sample = m->trace_on && (t % kTraceEvery == 0);
     for (int l = 0; l < M; ++l) {
-        if ((rc = lm_gemv<kLmStore>(pdl, m->Win + (size_t)l * 3 * D * D, 3 * D, D, m->u, B, 1, m->z, st))) return rc;
+        if ((rc = lm_gemv<kLmStore, 1, 2>(pdl, c->nsm, m->Win + (size_t)l * 3 * D * D, 3 * D, D, m->u, B, 1, m->z, nullptr, st))) return rc;
         const int e0 = sample ? lm_event(m, st) : -1;
         if ((rc = lm_launch(pdl, k_lm_mixer, dim3((B * D + 127) / 128), dim3(128), 0, st, (const float*)m->z,
                             m->zr + (size_t)l * 2 * B * 3 * D, (const float*)(m->conv + (size_t)l * 9 * D),
@@ -1401,14 +1429,15 @@ int lm_token(fi_lm* m, long long t, const int* tok_src, float* logits_out, int* 
                             c->yout + (size_t)l * G * L, m->u, (const TokIO*)io)))
             return rc;
         if (sample) m->ev_steps.push_back({e0, lm_event(m, st)});
-        if ((rc = lm_gemv<kLmGelu>(pdl, m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->u, B, 1, m->m1, st))) return rc;
-        if ((rc = lm_gemv<kLmAdd>(pdl, m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, st))) return rc;
+        if ((rc = lm_gemv<kLmGelu, 1, 2>(pdl, c->nsm, m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->u, B, 1, m->m1, nullptr, st))) return rc;
+        if ((rc = lm_gemv<kLmAdd, 4, 2>(pdl, c->nsm, m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, nullptr, st))) return rc;
     }
-    float* lg = logits_out ? logits_out : m->logits;
-    if ((rc = lm_gemv<kLmStore>(pdl, m->Wlm, V, D, m->u, B, 1, lg, st))) return rc;
+    // the LM head stores the logits only when they are asked for; its epilogue folds
+    // every row into the greedy choice, which the pick kernel reads
+    if ((rc = lm_gemv<kLmArgmax, 1, 4>(pdl, c->nsm, m->Wlm, V, D, m->u, B, 1, logits_out, m->amax, st))) return rc;
     const bool block_follows = t + 1 < L;
-    if ((rc = lm_launch(pdl, k_lm_argmax, dim3(B), dim3(256), 0, st, (const float*)lg, V, m->tok, next_out, io,
-                        (io && !block_follows) ? 1 : 0)))
+    if ((rc = lm_launch(pdl, k_lm_pick, dim3(1), dim3(32), 0, st, (const unsigned long long*)m->amax, B, m->tok,
+                        next_out, io, (io && !block_follows) ? 1 : 0)))
         return rc;
     if (block_follows) {
         const int e0 = m->trace_on ? lm_event(m, st) : -1;
@@ -1557,7 +1586,7 @@ void lm_free(fi_lm* m) {
     cudaFree(m->z);
     cudaFree(m->zr);
     cudaFree(m->m1);
-    cudaFree(m->logits);
+    cudaFree(m->amax);
     cudaFree(m->tok);
     cudaFree(m->next);
     cudaFree(m->stage_i);
@@ -1580,9 +1609,9 @@ int lm_create_impl(fi_lm* m, const float* E, const float* Wlm, const float* Win,
     int rc = create_impl(c, filters);
     if (rc) return rc;
     if ((rc = dev_alloc(c, &c->yout, (size_t)M * c->G * c->L))) return rc;
-    CK(cudaFuncSetAttribute(k_lm_gemv<kLmStore>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax - 1024));
-    CK(cudaFuncSetAttribute(k_lm_gemv<kLmGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax - 1024));
-    CK(cudaFuncSetAttribute(k_lm_gemv<kLmAdd>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax - 1024));
+    if ((rc = lm_gemv_attrs<kLmStore, 1, 2>()) || (rc = lm_gemv_attrs<kLmGelu, 1, 2>()) ||
+        (rc = lm_gemv_attrs<kLmAdd, 4, 2>()) || (rc = lm_gemv_attrs<kLmArgmax, 1, 4>()))
+        return rc;
     const size_t DD = (size_t)D * D;
     if ((rc = lm_upload_bf16(m, E, (size_t)V * D, &m->E))) return rc;
     if ((rc = lm_upload_bf16(m, Wlm, (size_t)V * D, &m->Wlm))) return rc;
@@ -1595,9 +1624,9 @@ int lm_create_impl(fi_lm* m, const float* E, const float* Wlm, const float* Win,
     if ((rc = lm_alloc(m, &m->z, (size_t)B * 3 * D))) return rc;
     if ((rc = lm_alloc(m, &m->zr, (size_t)M * 2 * B * 3 * D))) return rc;
     if ((rc = lm_alloc(m, &m->m1, (size_t)B * 4 * D))) return rc;
-    if ((rc = lm_alloc(m, &m->logits, (size_t)B * V))) return rc;
     if ((rc = lm_alloc(m, &m->tok, (size_t)B))) return rc;
     if ((rc = lm_alloc(m, &m->next, (size_t)B))) return rc;
+    if ((rc = lm_alloc(m, &m->amax, (size_t)B))) return rc;
     CK(cudaDeviceSynchronize());
     return FI_OK;
 }

@@ -223,6 +223,31 @@ __global__ void __launch_bounds__(NT) k_tile_direct(TileArgs a0) {
     if (a.io && a.advance) tok_advance_if_last(a.io);
 }
 
+// The same sum for a small block (U <= 8): one thread per tile, operands in registers.
+// A tile then costs a few 32-byte sectors (U inputs, 2U taps, U outputs each within one
+// aligned run), where one CTA per tile would be almost all launch and barrier.
+template <int U>
+__global__ void __launch_bounds__(128) k_tile_direct_small(TileArgs a0) {
+    const TileArgs a = with_step(a0);
+    const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (item < a.count) {
+        const TilePtrs p = tile_ptrs(a, item);
+        float x[U], h[2 * U];
+#pragma unroll
+        for (int j = 0; j < U; ++j) x[j] = p.in[j];
+#pragma unroll
+        for (int k = 1; k < 2 * U; ++k) h[k] = __ldg(p.taps + k);
+#pragma unroll
+        for (int r = 0; r < U; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < U; ++j) acc = fmaf(x[j], h[U + r - j], acc);
+            p.out[r] = a.overwrite ? acc : p.out[r] + acc;
+        }
+    }
+    if (a.io && a.advance) tok_advance_if_last(a.io);
+}
+
 // ----------------------------------------------------------------- shared-memory FFT
 // In-place Stockham autosort FFT (forward, e^{-2 pi i k m / N}) of N = 2^LOGN
 // complex values in shared memory, radix-4 passes plus one radix-2 pass when LOGN

@@ -11,7 +11,8 @@
 //   y_t  = running sum of the blocks + h_0 x_t   (the red cell)        k_lm_mixer
 //   u   += qc y_t                                                      k_lm_mixer
 //   u   += W2 bf16(GELU(W1 bf16(LN(u))))                               k_lm_gemv x2
-// then logits = W_lm bf16(LN(u)) and the greedy next token (k_lm_argmax).  The gray
+// then logits = W_lm bf16(LN(u)) and the greedy next token (folded into the LM head's
+// epilogue, read by k_lm_pick).  The gray
 // blocks of the mixers (the long convolutions' history) are the block kernels of
 // fi_kernels.cuh over the mixer inputs x of every layer, written onto the running
 // sums y of the same layer.
@@ -26,11 +27,22 @@
 namespace fi {
 
 constexpr int kLmMaxB = 8;        // batch rows per launch
-constexpr int kLmThreads = 128;   // threads of the matrix-vector kernels (4 warps: small N still fills the SMs)
-constexpr int kLmUnroll = 4;      // 16-byte weight loads a lane keeps in flight
+constexpr int kLmThreads = 256;   // threads of the matrix-vector kernels (8 warps; at most 2 CTAs an SM)
+constexpr int kLmCtasPerSm = 2;   // matrix-vector grid: one wave, so the per-CTA set-up (inputs, statistics) is paid once an SM slot
+constexpr int kLmUnroll = 3;      // 16-byte weight loads a lane keeps in flight per row (a 768-value slice: all of it)
 constexpr float kLmLnEps = 1e-5f;
 
-enum LmEpilogue { kLmStore = 0, kLmGelu = 1, kLmAdd = 2 };
+enum LmEpilogue { kLmStore = 0, kLmGelu = 1, kLmAdd = 2, kLmArgmax = 3 };
+
+// Greedy choice folded into the LM head: a logit and its id as one 64-bit key whose
+// unsigned order is the order of (logit, -id), so the maximum key over a row is its
+// largest logit with the lowest id among equal maxima.
+__device__ __forceinline__ unsigned long long lm_key(float v, int id) {
+    const unsigned u = __float_as_uint(v);
+    const unsigned o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)o << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned)id);
+}
+__device__ __forceinline__ int lm_key_id(unsigned long long k) { return (int)(0xFFFFFFFFu - (unsigned)(k & 0xFFFFFFFFull)); }
 
 // u[b][:] = E[tok[b]][:] (bf16 embedding rows to fp32)
 //
@@ -41,127 +53,238 @@ enum LmEpilogue { kLmStore = 0, kLmGelu = 1, kLmAdd = 2 };
 // waiting CTAs crowd the running kernel.  Reads of data another kernel writes go
 // through L2 only (ld.global.cg), which stays correct however the launches overlap.
 __global__ void k_lm_embed(const __nv_bfloat16* __restrict__ E, const int* __restrict__ tok, int B, int D,
-                           float* __restrict__ u) {
-    grid_dep_launch();
+                           float* __restrict__ u, unsigned long long* amax) {
     grid_dep_wait();
+    grid_dep_launch();
+    if (blockIdx.x == 0 && threadIdx.x < B) amax[threadIdx.x] = 0ull;  // this token's greedy choice starts empty
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < B * D; e += gridDim.x * blockDim.x) {
         const int b = e / D, d = e - b * D;
         u[e] = __bfloat162float(E[(long long)__ldcg(tok + b) * D + d]);
     }
 }
 
-// y[b][n] (epilogue)= sum_k W[n][k] bf16(pre(x[b][k])), n < N, b < B; pre = layer norm
-// over the row (ln = 1) or the identity.  Each warp takes rows n = warp + j * warps
-// (grid-stride over the launch); the B input rows, normalised and rounded to bf16, sit in
-// shared memory as fp32.  Epilogue: store, GELU then store, or add onto y (residual).
-template <int EPI>
-__global__ void __launch_bounds__(kLmThreads) k_lm_gemv(const __nv_bfloat16* __restrict__ W, int N, int K,
-                                                        const float* __restrict__ x, int B, int ln,
-                                                        float* __restrict__ y) {
-    extern __shared__ float xs[];  // [B][K]
-    __shared__ float stat[kLmMaxB][2];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = kLmThreads / 32;
-    grid_dep_launch();
+// y[b][n] (epilogue)= sum_k W[n][k] a[b][k], n < N, b < B, where a = bf16(LN(x)) (ln = 1)
+// or a = x, whose values are bf16 already (ln = 0: the GELU epilogue stores them so).
+//
+// Weight rows are read with 16-byte loads (8 bf16), lanes striding over a row.  A warp
+// takes RPW rows at a time, all their loads issued before any is used; with KS > 1
+// each row is split over KS warps, each summing a K / KS slice, the partial sums joined
+// in shared memory.  The B input rows a sit in shared memory as fp32 in two planes, the
+// first and second four values of every group of eight: the eight inputs matching a
+// lane's weight load are then one 16-byte read in each plane, consecutive lanes reading
+// consecutive 16 bytes (no bank conflicts), and each read serves all RPW rows.
+// Epilogue: store; GELU, rounded to bf16 (the next product's operand), then store; add
+// onto y (residual); or store (when y is given) and fold the row into the greedy choice
+// (amax[b], keys of lm_key).  BM >= B bounds the batch rows at compile time (4 or 8):
+// the accumulators of a warp are RPW x BM registers.
+template <int EPI, int KS, int RPW, int BM>
+__global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv_bfloat16* __restrict__ W, int N,
+                                                                     int K, const float* __restrict__ x, int B,
+                                                                     int ln, float* __restrict__ y,
+                                                                     unsigned long long* amax) {
+    extern __shared__ float xs[];  // planes [2][B][K / 2]
+    __shared__ float part[kLmThreads / 32][RPW][BM];
+    constexpr int nw = kLmThreads / 32;
+    constexpr int RPC = (nw / KS) * RPW;  // rows per CTA per step
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KH = K / 2, K8 = K / 8;
     // this CTA's weight rows into L2 (128-byte lines), before waiting for the input
     {
         const int lines = K * 2 / 128;  // whole 128-byte lines of a row (a partial last one is left out)
-        for (int n0 = blockIdx.x * nw; n0 < N; n0 += gridDim.x * nw) {
-            const int rows = min(nw, N - n0);
+        for (int n0 = blockIdx.x * RPC; n0 < N; n0 += gridDim.x * RPC) {
+            const int rows = min(RPC, N - n0);
             const char* base = reinterpret_cast<const char*>(W + (long long)n0 * K);
             for (int i = threadIdx.x; i < rows * lines; i += kLmThreads)
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (long long)i * 128));
         }
     }
     grid_dep_wait();
-    for (int e = threadIdx.x; e < B * K; e += kLmThreads) xs[e] = __ldcg(x + e);
+    grid_dep_launch();
+    {
+        // the inputs into the two planes, eight 16-byte loads a thread in flight at once
+        const float4* x4 = reinterpret_cast<const float4*>(x);
+        float4* xs4 = reinterpret_cast<float4*>(xs);
+        const int n4 = B * K / 4, K4 = K / 4;
+        for (int e0 = threadIdx.x; e0 < n4; e0 += 8 * kLmThreads) {
+            float4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (e0 + i * kLmThreads < n4) v[i] = __ldcg(x4 + e0 + i * kLmThreads);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int e = e0 + i * kLmThreads;
+                if (e < n4) {
+                    const int b = e / K4, q = e - b * K4;  // q: the 4-group within the row
+                    xs4[(q & 1) * (B * K8) + b * K8 + (q >> 1)] = v[i];
+                }
+            }
+        }
+    }
     __syncthreads();
     if (ln) {
-        // mean and variance of row b by warp b (two passes over shared memory)
+        // warp b normalises row b: mean, then variance about it (two passes), then
+        // bf16((x - mean) / sqrt(var + eps)); row b is the KH values at xs[b KH] and at
+        // xs[B KH + b KH], read as float4 (KH = K / 2 is a multiple of 4)
+        const int KQ = KH / 4;
         for (int b = warp; b < B; b += nw) {
+            float4* p0 = reinterpret_cast<float4*>(xs + b * KH);
+            float4* p1 = reinterpret_cast<float4*>(xs + B * KH + b * KH);
             float s = 0.f;
-            for (int k = lane; k < K; k += 32) s += xs[b * K + k];
+            for (int i = lane; i < KQ; i += 32) {
+                const float4 a = p0[i], c = p1[i];
+                s += ((a.x + a.y) + (a.z + a.w)) + ((c.x + c.y) + (c.z + c.w));
+            }
 #pragma unroll
             for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
             const float mean = s / (float)K;
             float v = 0.f;
-            for (int k = lane; k < K; k += 32) {
-                const float d = xs[b * K + k] - mean;
-                v = fmaf(d, d, v);
+            for (int i = lane; i < KQ; i += 32) {
+                const float4 a = p0[i], c = p1[i];
+                v = fmaf(a.x - mean, a.x - mean, v);
+                v = fmaf(a.y - mean, a.y - mean, v);
+                v = fmaf(a.z - mean, a.z - mean, v);
+                v = fmaf(a.w - mean, a.w - mean, v);
+                v = fmaf(c.x - mean, c.x - mean, v);
+                v = fmaf(c.y - mean, c.y - mean, v);
+                v = fmaf(c.z - mean, c.z - mean, v);
+                v = fmaf(c.w - mean, c.w - mean, v);
             }
 #pragma unroll
             for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) {
-                stat[b][0] = mean;
-                stat[b][1] = 1.0f / sqrtf(v / (float)K + kLmLnEps);
+            const float rstd = 1.0f / sqrtf(v / (float)K + kLmLnEps);
+            auto nrm = [&](float t) { return __bfloat162float(__float2bfloat16_rn((t - mean) * rstd)); };
+            for (int i = lane; i < KQ; i += 32) {
+                float4 a = p0[i], c = p1[i];
+                a = make_float4(nrm(a.x), nrm(a.y), nrm(a.z), nrm(a.w));
+                c = make_float4(nrm(c.x), nrm(c.y), nrm(c.z), nrm(c.w));
+                p0[i] = a;
+                p1[i] = c;
             }
         }
         __syncthreads();
     }
-    for (int e = threadIdx.x; e < B * K; e += kLmThreads) {
-        const int b = e / K;
-        const float v = ln ? (xs[e] - stat[b][0]) * stat[b][1] : xs[e];
-        xs[e] = __bfloat162float(__float2bfloat16_rn(v));
-    }
-    __syncthreads();
-    // rows: 8 bf16 weights per 16-byte load, lanes stride over the row, kLmUnroll loads
-    // in flight per lane before they are used
-    const int K8 = K / 8;
-    for (int n = blockIdx.x * nw + warp; n < N; n += gridDim.x * nw) {
-        const uint4* wr = reinterpret_cast<const uint4*>(W + (long long)n * K);
-        float acc[kLmMaxB];
+    const float4* xlo = reinterpret_cast<const float4*>(xs);
+    const float4* xhi = xlo + B * K8;
+    const int Kw = K / KS;  // this warp's slice of a row
+    const int j0 = (KS > 1 ? warp % KS : 0) * (Kw / 8);
+    const int S8 = Kw / 8;
+    // greedy choice: each writing warp's running best per batch row (lane 0 owns it)
+    __shared__ unsigned long long sbest[nw][BM];
+    if (EPI == kLmArgmax && lane == 0)
 #pragma unroll
-        for (int b = 0; b < kLmMaxB; ++b) acc[b] = 0.f;
-        for (int v0 = lane; v0 < K8; v0 += 32 * kLmUnroll) {
-            uint4 pk[kLmUnroll];
+        for (int b = 0; b < BM; ++b) sbest[warp][b] = 0ull;
+    for (int n0 = blockIdx.x * RPC; n0 < N; n0 += gridDim.x * RPC) {
+        int rows[RPW];
 #pragma unroll
-            for (int u = 0; u < kLmUnroll; ++u) {
-                const int v8 = v0 + 32 * u;
-                pk[u] = v8 < K8 ? __ldg(wr + v8) : make_uint4(0u, 0u, 0u, 0u);
+        for (int r = 0; r < RPW; ++r) rows[r] = n0 + (warp / KS) * RPW + r;
+        float acc[RPW][BM];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int b = 0; b < BM; ++b) acc[r][b] = 0.f;
+        for (int v0 = lane; v0 < S8; v0 += 32 * kLmUnroll) {
+            uint4 pk[RPW][kLmUnroll];
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) {
+                const uint4* wr = reinterpret_cast<const uint4*>(W + (long long)min(rows[r], N - 1) * K) + j0;
+#pragma unroll
+                for (int u = 0; u < kLmUnroll; ++u) {
+                    const int v8 = v0 + 32 * u;
+                    pk[r][u] = (v8 < S8 && rows[r] < N) ? __ldg(wr + v8) : make_uint4(0u, 0u, 0u, 0u);
+                }
             }
 #pragma unroll
             for (int u = 0; u < kLmUnroll; ++u) {
                 const int v8 = v0 + 32 * u;
-                if (v8 < K8) {
-                    const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&pk[u]);
-                    float w[8];
+                if (v8 < S8) {
+                    float w[RPW][8];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = __bfloat1622float2(w2[i]);
-                        w[2 * i] = f.x;
-                        w[2 * i + 1] = f.y;
+                    for (int r = 0; r < RPW; ++r) {
+                        const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&pk[r][u]);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = __bfloat1622float2(w2[i]);
+                            w[r][2 * i] = f.x;
+                            w[r][2 * i + 1] = f.y;
+                        }
                     }
 #pragma unroll
-                    for (int b = 0; b < kLmMaxB; ++b) {
+                    for (int b = 0; b < BM; ++b) {
                         if (b < B) {
-                            const float4* xr = reinterpret_cast<const float4*>(xs + b * K + 8 * v8);
-                            const float4 x0 = xr[0], x1 = xr[1];
-                            float a = acc[b];
-                            a = fmaf(w[0], x0.x, a);
-                            a = fmaf(w[1], x0.y, a);
-                            a = fmaf(w[2], x0.z, a);
-                            a = fmaf(w[3], x0.w, a);
-                            a = fmaf(w[4], x1.x, a);
-                            a = fmaf(w[5], x1.y, a);
-                            a = fmaf(w[6], x1.z, a);
-                            a = fmaf(w[7], x1.w, a);
-                            acc[b] = a;
+                            const float4 x0 = xlo[b * K8 + j0 + v8], x1 = xhi[b * K8 + j0 + v8];
+#pragma unroll
+                            for (int r = 0; r < RPW; ++r) {
+                                float a = acc[r][b];
+                                a = fmaf(w[r][0], x0.x, a);
+                                a = fmaf(w[r][1], x0.y, a);
+                                a = fmaf(w[r][2], x0.z, a);
+                                a = fmaf(w[r][3], x0.w, a);
+                                a = fmaf(w[r][4], x1.x, a);
+                                a = fmaf(w[r][5], x1.y, a);
+                                a = fmaf(w[r][6], x1.z, a);
+                                a = fmaf(w[r][7], x1.w, a);
+                                acc[r][b] = a;
+                            }
                         }
                     }
                 }
             }
         }
+        // sums over the lanes (every lane ends with all of them); lane (rl, bl) = (lane /
+        // BM, lane % BM) then finishes row rl of the step for batch row bl; with KS > 1
+        // the writing warp adds the partial sums of the warps sharing its rows
 #pragma unroll
-        for (int b = 0; b < kLmMaxB; ++b) {
-            if (b < B) {
-                float a = acc[b];
+        for (int r = 0; r < RPW; ++r)
 #pragma unroll
-                for (int o = 16; o; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-                if (lane == 0) {
-                    if (EPI == kLmGelu) a = 0.5f * a * (1.0f + erff(a * 0.70710678118654752f));
-                    if (EPI == kLmAdd) y[(long long)b * N + n] = __ldcg(y + (long long)b * N + n) + a;
-                    else y[(long long)b * N + n] = a;
+            for (int b = 0; b < BM; ++b)
+                if (b < B) {
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) acc[r][b] += __shfl_xor_sync(0xffffffffu, acc[r][b], o);
                 }
+        const int rl = lane / BM, bl = lane % BM;
+        float a = 0.f;
+#pragma unroll
+        for (int r = 0; r < RPW; ++r)
+#pragma unroll
+            for (int b = 0; b < BM; ++b)
+                if (r == rl && b == bl) a = acc[r][b];
+        const bool pair = rl < RPW && bl < B;
+        if (KS > 1) {
+            if (pair) part[warp][rl][bl] = a;
+            __syncthreads();
+            if (warp % KS == 0 && pair) {
+                a = 0.f;
+                for (int w = 0; w < KS; ++w) a += part[warp + w][rl][bl];
             }
+            __syncthreads();
+        }
+        const bool writer = KS == 1 || warp % KS == 0;
+        const int n = n0 + (warp / KS) * RPW + rl;
+        const bool own = writer && pair && n < N;
+        if (own) {
+            if (EPI == kLmGelu) a = __bfloat162float(__float2bfloat16_rn(0.5f * a * (1.0f + erff(a * 0.70710678118654752f))));
+            if (EPI == kLmAdd) y[(long long)bl * N + n] = __ldcg(y + (long long)bl * N + n) + a;
+            else if (EPI != kLmArgmax || y) y[(long long)bl * N + n] = a;
+        }
+        if (EPI == kLmArgmax) {
+            // the step's best per batch row: a maximum over the lanes of equal bl
+            unsigned long long k = own ? lm_key(a, n) : 0ull;
+#pragma unroll
+            for (int o = BM; o < RPW * BM; o <<= 1) {
+                const unsigned long long q = __shfl_xor_sync(0xffffffffu, k, o);
+                k = q > k ? q : k;
+            }
+            if (writer && rl == 0 && bl < B && k > sbest[warp][bl]) sbest[warp][bl] = k;
+        }
+    }
+    if (EPI == kLmArgmax) {
+        // the CTA's best per row, then one atomic per row and CTA
+        __syncthreads();
+        if (threadIdx.x < B) {
+            unsigned long long k = 0ull;
+#pragma unroll
+            for (int w = 0; w < nw; ++w) k = sbest[w][threadIdx.x] > k ? sbest[w][threadIdx.x] : k;
+            if (k) atomicMax(amax + threadIdx.x, k);
         }
     }
 }
@@ -176,76 +299,57 @@ __global__ void k_lm_mixer(const float* __restrict__ z, float* __restrict__ zr, 
                            const float* __restrict__ h, long long L, int B, int D, long long t, float* X,
                            float* Y, float* u, const TokIO* io) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
-    grid_dep_launch();
     grid_dep_wait();
-    if (io) t = io->t;
+    grid_dep_launch();
     if (e >= B * D) return;
     const int b = e / D, d = e - b * D;
     const int D3 = 3 * D;
-    float zc[3];
+    // every load first (one round trip), then the arithmetic and the stores
+    float z0[3], z1[3], z2[3], c0[3], c1[3], c2[3];
+    float* r1 = zr + (long long)b * D3 + d;                      // z_{t-1}
+    float* r2 = zr + (long long)B * D3 + (long long)b * D3 + d;  // z_{t-2}
 #pragma unroll
     for (int s = 0; s < 3; ++s) {
         const int j = s * D + d;
-        const float z0 = __ldcg(z + b * D3 + j);
-        float* r1 = zr + (long long)b * D3 + j;                 // z_{t-1}
-        float* r2 = zr + (long long)B * D3 + (long long)b * D3 + j;  // z_{t-2}
-        const float z1 = __ldcg(r1), z2 = __ldcg(r2);
-        zc[s] = fmaf(conv[j], z0, fmaf(conv[D3 + j], z1, conv[2 * D3 + j] * z2));
-        *r2 = z1;
-        *r1 = z0;
+        z0[s] = __ldcg(z + b * D3 + j);
+        z1[s] = __ldcg(r1 + s * D);
+        z2[s] = __ldcg(r2 + s * D);
+        c0[s] = __ldg(conv + j);
+        c1[s] = __ldg(conv + D3 + j);
+        c2[s] = __ldg(conv + 2 * D3 + j);
+    }
+    const float h0 = __ldg(h + (long long)d * L);
+    const float u0 = __ldcg(u + e);
+    if (io) t = io->t;
+    const long long g = (long long)b * D + d;
+    const float run = t == 0 ? 0.f : __ldcg(Y + g * L + t);
+    float zc[3];
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        zc[s] = fmaf(c0[s], z0[s], fmaf(c1[s], z1[s], c2[s] * z2[s]));
+        r2[s * D] = z1[s];
+        r1[s * D] = z0[s];
     }
     const float x = zc[1] * zc[2];
-    const long long g = (long long)b * D + d;
     X[g * L + t] = x;
-    const float run = t == 0 ? 0.f : __ldcg(Y + g * L + t);
-    const float yv = fmaf(h[(long long)d * L], x, run);
+    const float yv = fmaf(h0, x, run);
     Y[g * L + t] = yv;
-    u[e] = fmaf(zc[0], yv, __ldcg(u + e));
+    u[e] = fmaf(zc[0], yv, u0);
 }
 
-// next[b] = argmax_v logits[b][v] (the lowest id among equal maxima), one CTA per row;
-// also written to out[b] when given, and used as the next input token.  With io (a
-// replayed per-token graph) out is the record's choice array at the record's token, and
-// with advance this launch closes the token.
-__global__ void k_lm_argmax(const float* __restrict__ logits, int V, int* next, int* out, TokIO* io, int advance) {
-    __shared__ float bv[32];
-    __shared__ int bi[32];
-    const int b = blockIdx.x;
-    grid_dep_launch();
+// next[b] = the greedy choice the LM head folded into amax[b] (largest logit, lowest id
+// among equal maxima); also written to out[b] when given, and used as the next input
+// token.  With io (a replayed per-token graph) out is the record's choice array at the
+// record's token, and with advance this launch closes the token.
+__global__ void k_lm_pick(const unsigned long long* __restrict__ amax, int B, int* next, int* out, TokIO* io,
+                          int advance) {
     grid_dep_wait();
-    const float* row = logits + (long long)b * V;
-    float best = -INFINITY;
-    int idx = 0x7fffffff;
-    for (int v = threadIdx.x; v < V; v += blockDim.x) {
-        const float x = __ldcg(row + v);
-        if (x > best || (x == best && v < idx)) {
-            best = x;
-            idx = v;
-        }
-    }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, idx, o);
-        if (ob > best || (ob == best && oi < idx)) {
-            best = ob;
-            idx = oi;
-        }
-    }
-    if (lane == 0) {
-        bv[warp] = best;
-        bi[warp] = idx;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
-            if (bv[w] > best || (bv[w] == best && bi[w] < idx)) {
-                best = bv[w];
-                idx = bi[w];
-            }
+    grid_dep_launch();
+    const int b = threadIdx.x;
+    if (b < B) {
+        const int idx = lm_key_id(__ldcg(amax + b));
         next[b] = idx;
-        if (io) out = io->itok + (io->t - io->tx) * gridDim.x;
+        if (io) out = io->itok + (io->t - io->tx) * B;
         if (out) out[b] = idx;
     }
     if (io && advance) tok_advance_if_last(io);
