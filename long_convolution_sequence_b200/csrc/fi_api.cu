@@ -1285,6 +1285,7 @@ struct fi_lm {
     __nv_bfloat16 *E = nullptr, *Wlm = nullptr, *Win = nullptr, *W1 = nullptr, *W2 = nullptr;
     float* conv = nullptr;                       // [M][3][3D]
     float *u = nullptr, *z = nullptr, *zr = nullptr, *m1 = nullptr;
+    float* r = nullptr;                          // [B][D]: u + qc y_t, the MLP's input and residual
     int *tok = nullptr, *next = nullptr;         // [B]: the next input token, the latest choice
     unsigned long long* amax = nullptr;          // [B]: the LM head's running greedy choice (keys of lm_key)
     int* stage_i = nullptr;                      // host token arrays staged on the device
@@ -1381,15 +1382,17 @@ int lm_launch(int pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // inputs serves two or four rows.  At most kLmCtasPerSm CTAs an SM (one wave).
 template <int EPI, int KS, int RPW>
 int lm_gemv(int pdl, int nsm, const __nv_bfloat16* W, int N, int K, const float* x, int B, int ln, float* y,
-            unsigned long long* amax, cudaStream_t st) {
-    const int rows_per_cta = ((kLmThreads / 32) / KS) * RPW;
-    const int grid = std::min((N + rows_per_cta - 1) / rows_per_cta, kLmCtasPerSm * nsm);
+            const LmEpi& ep, cudaStream_t st) {
+    // units: rows, or (mixer epilogue) channels, one a warp
+    const int units = EPI == kLmMix ? ep.D : N;
+    const int per_cta = EPI == kLmMix ? (kLmThreads / 32) / KS : ((kLmThreads / 32) / KS) * RPW;
+    const int grid = std::min((units + per_cta - 1) / per_cta, kLmCtasPerSm * nsm);
     const size_t smem = (size_t)B * K * sizeof(float);
     if (B <= 4)
         return lm_launch(pdl, k_lm_gemv<EPI, KS, RPW, 4>, dim3(grid), dim3(kLmThreads), smem, st, W, N, K, x, B, ln, y,
-                         amax);
+                         ep);
     return lm_launch(pdl, k_lm_gemv<EPI, KS, RPW, kLmMaxB>, dim3(grid), dim3(kLmThreads), smem, st, W, N, K, x, B, ln,
-                     y, amax);
+                     y, ep);
 }
 
 template <int EPI, int KS, int RPW>
@@ -1420,21 +1423,52 @@ int lm_token(fi_lm* m, long long t, const int* tok_src, float* logits_out, int* 
                         tok_src, B, D, m->u, m->amax)))
         return rc;
     const bool sample = m->trace_on && (t % kTraceEvery == 0);
+    const LmEpi none = {};
     for (int l = 0; l < M; ++l) {
-        if ((rc = lm_gemv<kLmStore, 1, 2>(pdl, c->nsm, m->Win + (size_t)l * 3 * D * D, 3 * D, D, m->u, B, 1, m->z, nullptr, st))) return rc;
-        const int e0 = sample ? lm_event(m, st) : -1;
-        if ((rc = lm_launch(pdl, k_lm_mixer, dim3((B * D + 127) / 128), dim3(128), 0, st, (const float*)m->z,
-                            m->zr + (size_t)l * 2 * B * 3 * D, (const float*)(m->conv + (size_t)l * 9 * D),
-                            (const float*)(c->h + (size_t)l * D * L), L, B, D, t, c->act + (size_t)l * G * L,
-                            c->yout + (size_t)l * G * L, m->u, (const TokIO*)io)))
+        // in-projection and mixer step: r = u + qc y_t (fused; traced runs launch the
+        // mixer step on its own, to time it)
+        LmEpi mx = {};
+        mx.zr = m->zr + (size_t)l * 2 * B * 3 * D;
+        mx.conv = m->conv + (size_t)l * 9 * D;
+        mx.h = c->h + (size_t)l * D * L;
+        mx.L = L;
+        mx.t = t;
+        mx.X = c->act + (size_t)l * G * L;
+        mx.Y = c->yout + (size_t)l * G * L;
+        mx.io = io;
+        mx.D = D;
+        const __nv_bfloat16* Win = m->Win + (size_t)l * 3 * D * D;
+        if (!m->trace_on) {
+            // a channel's three rows split over two warps (16-byte slices need D % 16 == 0)
+            rc = (D % 16 == 0) ? lm_gemv<kLmMix, 2, 3>(pdl, c->nsm, Win, 3 * D, D, m->u, B, 1, m->r, mx, st)
+                               : lm_gemv<kLmMix, 1, 3>(pdl, c->nsm, Win, 3 * D, D, m->u, B, 1, m->r, mx, st);
+            if (rc) return rc;
+        } else {
+            // the same row split as the fused kernel: the same sums, bit for bit
+            rc = (D % 16 == 0) ? lm_gemv<kLmStore, 2, 2>(pdl, c->nsm, Win, 3 * D, D, m->u, B, 1, m->z, none, st)
+                               : lm_gemv<kLmStore, 1, 2>(pdl, c->nsm, Win, 3 * D, D, m->u, B, 1, m->z, none, st);
+            if (rc) return rc;
+            const int e0 = sample ? lm_event(m, st) : -1;
+            if ((rc = lm_launch(pdl, k_lm_mixer, dim3((B * D + 127) / 128), dim3(128), 0, st, (const float*)m->z, mx.zr,
+                                mx.conv, mx.h, L, B, D, t, mx.X, mx.Y, (const float*)m->u, m->r, (const TokIO*)io)))
+                return rc;
+            if (sample) m->ev_steps.push_back({e0, lm_event(m, st)});
+        }
+        // MLP: u = r + W2 bf16(GELU(W1 bf16(LN(r))))
+        if ((rc = lm_gemv<kLmGelu, 1, 2>(pdl, c->nsm, m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->r, B, 1, m->m1, none,
+                                         st)))
             return rc;
-        if (sample) m->ev_steps.push_back({e0, lm_event(m, st)});
-        if ((rc = lm_gemv<kLmGelu, 1, 2>(pdl, c->nsm, m->W1 + (size_t)l * 4 * D * D, 4 * D, D, m->u, B, 1, m->m1, nullptr, st))) return rc;
-        if ((rc = lm_gemv<kLmAdd, 4, 2>(pdl, c->nsm, m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, nullptr, st))) return rc;
+        LmEpi ad = {};
+        ad.res = m->r;
+        if ((rc = lm_gemv<kLmAdd, 4, 2>(pdl, c->nsm, m->W2 + (size_t)l * 4 * D * D, D, 4 * D, m->m1, B, 0, m->u, ad,
+                                        st)))
+            return rc;
     }
     // the LM head stores the logits only when they are asked for; its epilogue folds
     // every row into the greedy choice, which the pick kernel reads
-    if ((rc = lm_gemv<kLmArgmax, 1, 4>(pdl, c->nsm, m->Wlm, V, D, m->u, B, 1, logits_out, m->amax, st))) return rc;
+    LmEpi hd = {};
+    hd.amax = m->amax;
+    if ((rc = lm_gemv<kLmArgmax, 1, 4>(pdl, c->nsm, m->Wlm, V, D, m->u, B, 1, logits_out, hd, st))) return rc;
     const bool block_follows = t + 1 < L;
     if ((rc = lm_launch(pdl, k_lm_pick, dim3(1), dim3(32), 0, st, (const unsigned long long*)m->amax, B, m->tok,
                         next_out, io, (io && !block_follows) ? 1 : 0)))
@@ -1586,6 +1620,7 @@ void lm_free(fi_lm* m) {
     cudaFree(m->z);
     cudaFree(m->zr);
     cudaFree(m->m1);
+    cudaFree(m->r);
     cudaFree(m->amax);
     cudaFree(m->tok);
     cudaFree(m->next);
@@ -1609,8 +1644,9 @@ int lm_create_impl(fi_lm* m, const float* E, const float* Wlm, const float* Win,
     int rc = create_impl(c, filters);
     if (rc) return rc;
     if ((rc = dev_alloc(c, &c->yout, (size_t)M * c->G * c->L))) return rc;
-    if ((rc = lm_gemv_attrs<kLmStore, 1, 2>()) || (rc = lm_gemv_attrs<kLmGelu, 1, 2>()) ||
-        (rc = lm_gemv_attrs<kLmAdd, 4, 2>()) || (rc = lm_gemv_attrs<kLmArgmax, 1, 4>()))
+    if ((rc = lm_gemv_attrs<kLmStore, 1, 2>()) || (rc = lm_gemv_attrs<kLmStore, 2, 2>()) || (rc = lm_gemv_attrs<kLmMix, 1, 3>()) || (rc = lm_gemv_attrs<kLmMix, 2, 3>()) ||
+        (rc = lm_gemv_attrs<kLmGelu, 1, 2>()) || (rc = lm_gemv_attrs<kLmAdd, 4, 2>()) ||
+        (rc = lm_gemv_attrs<kLmArgmax, 1, 4>()))
         return rc;
     const size_t DD = (size_t)D * D;
     if ((rc = lm_upload_bf16(m, E, (size_t)V * D, &m->E))) return rc;
@@ -1624,6 +1660,7 @@ int lm_create_impl(fi_lm* m, const float* E, const float* Wlm, const float* Win,
     if ((rc = lm_alloc(m, &m->z, (size_t)B * 3 * D))) return rc;
     if ((rc = lm_alloc(m, &m->zr, (size_t)M * 2 * B * 3 * D))) return rc;
     if ((rc = lm_alloc(m, &m->m1, (size_t)B * 4 * D))) return rc;
+    if ((rc = lm_alloc(m, &m->r, (size_t)B * D))) return rc;
     if ((rc = lm_alloc(m, &m->tok, (size_t)B))) return rc;
     if ((rc = lm_alloc(m, &m->next, (size_t)B))) return rc;
     if ((rc = lm_alloc(m, &m->amax, (size_t)B))) return rc;

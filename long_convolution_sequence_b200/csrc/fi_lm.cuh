@@ -32,7 +32,7 @@ constexpr int kLmCtasPerSm = 2;   // matrix-vector grid: one wave, so the per-CT
 constexpr int kLmUnroll = 3;      // 16-byte weight loads a lane keeps in flight per row (a 768-value slice: all of it)
 constexpr float kLmLnEps = 1e-5f;
 
-enum LmEpilogue { kLmStore = 0, kLmGelu = 1, kLmAdd = 2, kLmArgmax = 3 };
+enum LmEpilogue { kLmStore = 0, kLmGelu = 1, kLmAdd = 2, kLmArgmax = 3, kLmMix = 4 };
 
 // Greedy choice folded into the LM head: a logit and its id as one 64-bit key whose
 // unsigned order is the order of (logit, -id), so the maximum key over a row is its
@@ -63,55 +63,176 @@ __global__ void k_lm_embed(const __nv_bfloat16* __restrict__ E, const int* __res
     }
 }
 
+// The mixer part of layer l at token t for batch row b and channel d, given the
+// in-projection's q, k, v values of the token: short convolution of the three streams
+// with the two previous tokens' values (ring zr[2][B][3D], shifted here), the gate
+// x = kc vc stored as the mixer's input at t, the red cell y_t = (running sum at t) +
+// h_0 x_t (the running sum is 0 at t = 0, where no block has written), y_t kept at t,
+// and the gated residual r = u + qc y_t.  Its loads (MixOps) do not depend on q, k, v
+// and are issued first.
+struct MixOps {
+    float z1[3], z2[3], c0[3], c1[3], c2[3];
+    float h0, u0, run;
+};
+
+__device__ __forceinline__ MixOps lm_mixer_load(int b, int d, const float* zr, const float* __restrict__ conv,
+                                                const float* __restrict__ h, long long L, int B, int D, long long t,
+                                                const float* Y, const float* u) {
+    MixOps o;
+    const int D3 = 3 * D;
+    const float* r1 = zr + (long long)b * D3 + d;                      // z_{t-1}
+    const float* r2 = zr + (long long)B * D3 + (long long)b * D3 + d;  // z_{t-2}
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        const int j = s * D + d;
+        o.z1[s] = __ldcg(r1 + s * D);
+        o.z2[s] = __ldcg(r2 + s * D);
+        o.c0[s] = __ldg(conv + j);
+        o.c1[s] = __ldg(conv + D3 + j);
+        o.c2[s] = __ldg(conv + 2 * D3 + j);
+    }
+    o.h0 = __ldg(h + (long long)d * L);
+    const long long g = (long long)b * D + d;
+    o.u0 = __ldcg(u + g);
+    o.run = t == 0 ? 0.f : __ldcg(Y + g * L + t);
+    return o;
+}
+
+__device__ __forceinline__ void lm_mixer_finish(const MixOps& o, float zq, float zk, float zv, int b, int d,
+                                                float* zr, long long L, int B, int D, long long t, float* X, float* Y,
+                                                float* r) {
+    const int D3 = 3 * D;
+    const float z0[3] = {zq, zk, zv};
+    float* r1 = zr + (long long)b * D3 + d;
+    float* r2 = zr + (long long)B * D3 + (long long)b * D3 + d;
+    float zc[3];
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        zc[s] = fmaf(o.c0[s], z0[s], fmaf(o.c1[s], o.z1[s], o.c2[s] * o.z2[s]));
+        r2[s * D] = o.z1[s];
+        r1[s * D] = z0[s];
+    }
+    const long long g = (long long)b * D + d;
+    const float xv = zc[1] * zc[2];
+    X[g * L + t] = xv;
+    const float yv = fmaf(o.h0, xv, o.run);
+    Y[g * L + t] = yv;
+    r[g] = fmaf(zc[0], yv, o.u0);
+}
+
+// Epilogue operands of the matrix-vector kernel beyond y.
+struct LmEpi {
+    unsigned long long* amax;  // kLmArgmax: running greedy choice per batch row
+    const float* res;          // kLmAdd: y = res + W x (res may be y)
+    // kLmMix: the mixer step of the layer (as k_lm_mixer), u the kernel's input x
+    float* zr;
+    const float* conv;
+    const float* h;
+    long long L;
+    long long t;
+    float* X;
+    float* Y;
+    const TokIO* io;
+    int D;
+};
+
 // y[b][n] (epilogue)= sum_k W[n][k] a[b][k], n < N, b < B, where a = bf16(LN(x)) (ln = 1)
 // or a = x, whose values are bf16 already (ln = 0: the GELU epilogue stores them so).
 //
 // Weight rows are read with 16-byte loads (8 bf16), lanes striding over a row.  A warp
-// takes RPW rows at a time, all their loads issued before any is used; with KS > 1
-// each row is split over KS warps, each summing a K / KS slice, the partial sums joined
-// in shared memory.  The B input rows a sit in shared memory as fp32 in two planes, the
-// first and second four values of every group of eight: the eight inputs matching a
-// lane's weight load are then one 16-byte read in each plane, consecutive lanes reading
-// consecutive 16 bytes (no bank conflicts), and each read serves all RPW rows.
-// Epilogue: store; GELU, rounded to bf16 (the next product's operand), then store; add
-// onto y (residual); or store (when y is given) and fold the row into the greedy choice
-// (amax[b], keys of lm_key).  BM >= B bounds the batch rows at compile time (4 or 8):
-// the accumulators of a warp are RPW x BM registers.
+// takes RPW rows at a time, all their loads issued before any is used (the first step's
+// before the inputs are staged: they do not depend on them); with KS > 1 each row is
+// split over KS warps, each summing a K / KS slice, the partial sums joined in shared
+// memory.  The B input rows a sit in shared memory as fp32 in two planes, the first and
+// second four values of every group of eight: the eight inputs matching a lane's weight
+// load are then one 16-byte read in each plane, consecutive lanes reading consecutive 16
+// bytes (no bank conflicts), and each read serves all RPW rows.
+// Epilogue: store; GELU, rounded to bf16 (the next product's operand), then store;
+// y = res + W a (residual); store (when y is given) and fold the row into the greedy
+// choice (amax[b], keys of lm_key); or (kLmMix, RPW = 3) the mixer step: a warp takes
+// the rows d, D + d, 2D + d of the in-projection (q, k, v of channel d) and finishes
+// channel d as k_lm_mixer does, writing y = u + qc y_t (y is then not the input).
+// BM >= B bounds the batch rows at compile time (4 or 8): the accumulators of a warp
+// are RPW x BM registers.
 template <int EPI, int KS, int RPW, int BM>
 __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv_bfloat16* __restrict__ W, int N,
                                                                      int K, const float* __restrict__ x, int B,
-                                                                     int ln, float* __restrict__ y,
-                                                                     unsigned long long* amax) {
+                                                                     int ln, float* __restrict__ y, LmEpi ep) {
     extern __shared__ float xs[];  // planes [2][B][K / 2]
     __shared__ float part[kLmThreads / 32][RPW][BM];
     constexpr int nw = kLmThreads / 32;
-    constexpr int RPC = (nw / KS) * RPW;  // rows per CTA per step
+    constexpr bool MIX = EPI == kLmMix;
+    static_assert(!MIX || RPW == 3, "the mixer epilogue takes the q, k, v rows of a channel in one warp");
+    // units: rows, or (MIX) channels whose three rows KS warps share
+    constexpr int UPC = MIX ? nw / KS : (nw / KS) * RPW;  // units per CTA per step
+    const int NU = MIX ? ep.D : N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KH = K / 2, K8 = K / 8;
-    // this CTA's weight rows into L2 (128-byte lines), before waiting for the input
+    const int Kw = K / KS;  // this warp's slice of a row
+    const int j0 = (KS > 1 ? warp % KS : 0) * (Kw / 8);
+    const int S8 = Kw / 8;
+    auto row_of = [&](int u0, int r) -> int {  // weight row r of this warp at step u0, or -1
+        if (MIX) {
+            const int ch = u0 + warp / KS;
+            return ch < NU ? r * ep.D + ch : -1;
+        }
+        const int n = u0 + (warp / KS) * RPW + r;
+        return n < N ? n : -1;
+    };
+    uint4 pk[RPW][kLmUnroll];
+    auto load_w = [&](int u0, int v0) {
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+            const int n = row_of(u0, r);
+            const uint4* wr = reinterpret_cast<const uint4*>(W + (long long)max(n, 0) * K) + j0;
+#pragma unroll
+            for (int u = 0; u < kLmUnroll; ++u) {
+                const int v8 = v0 + 32 * u;
+                pk[r][u] = (v8 < S8 && n >= 0) ? __ldg(wr + v8) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    // the weight rows of this CTA into L2 (128-byte lines), and the first step's loads,
+    // before waiting for the input
     {
         const int lines = K * 2 / 128;  // whole 128-byte lines of a row (a partial last one is left out)
-        for (int n0 = blockIdx.x * RPC; n0 < N; n0 += gridDim.x * RPC) {
-            const int rows = min(RPC, N - n0);
-            const char* base = reinterpret_cast<const char*>(W + (long long)n0 * K);
-            for (int i = threadIdx.x; i < rows * lines; i += kLmThreads)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (long long)i * 128));
+        constexpr int nseg = MIX ? 3 : 1;
+        for (int u0 = blockIdx.x * UPC; u0 < NU; u0 += gridDim.x * UPC) {
+            const int units = min(UPC, NU - u0);
+            for (int sg = 0; sg < nseg; ++sg) {
+                const long long r0 = MIX ? (long long)sg * ep.D + u0 : u0;
+                const char* base = reinterpret_cast<const char*>(W + r0 * K);
+                for (int i = threadIdx.x; i < units * lines; i += kLmThreads)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (long long)i * 128));
+            }
         }
     }
+    load_w(blockIdx.x * UPC, lane);
     grid_dep_wait();
     grid_dep_launch();
+    // mixer epilogue: lane b < B of a channel's first warp finishes (b, channel); its
+    // operands for the first step are loaded now, in the shadow of the staging
+    long long t = ep.t;
+    MixOps mo;
+    const bool mix_lane = MIX && lane < B && (KS == 1 || warp % KS == 0);
+    if (MIX) {
+        if (ep.io) t = ep.io->t;
+        const int d = blockIdx.x * UPC + warp / KS;
+        if (mix_lane && d < NU) mo = lm_mixer_load(lane, d, ep.zr, ep.conv, ep.h, ep.L, B, ep.D, t, ep.Y, x);
+    }
     {
-        // the inputs into the two planes, eight 16-byte loads a thread in flight at once
+        // the inputs into the two planes, twelve 16-byte loads a thread in flight at once
+        constexpr int SB = 12;
         const float4* x4 = reinterpret_cast<const float4*>(x);
         float4* xs4 = reinterpret_cast<float4*>(xs);
         const int n4 = B * K / 4, K4 = K / 4;
-        for (int e0 = threadIdx.x; e0 < n4; e0 += 8 * kLmThreads) {
-            float4 v[8];
+        for (int e0 = threadIdx.x; e0 < n4; e0 += SB * kLmThreads) {
+            float4 v[SB];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int i = 0; i < SB; ++i)
                 if (e0 + i * kLmThreads < n4) v[i] = __ldcg(x4 + e0 + i * kLmThreads);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < SB; ++i) {
                 const int e = e0 + i * kLmThreads;
                 if (e < n4) {
                     const int b = e / K4, q = e - b * K4;  // q: the 4-group within the row
@@ -165,34 +286,21 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
     }
     const float4* xlo = reinterpret_cast<const float4*>(xs);
     const float4* xhi = xlo + B * K8;
-    const int Kw = K / KS;  // this warp's slice of a row
-    const int j0 = (KS > 1 ? warp % KS : 0) * (Kw / 8);
-    const int S8 = Kw / 8;
     // greedy choice: each writing warp's running best per batch row (lane 0 owns it)
     __shared__ unsigned long long sbest[nw][BM];
     if (EPI == kLmArgmax && lane == 0)
 #pragma unroll
         for (int b = 0; b < BM; ++b) sbest[warp][b] = 0ull;
-    for (int n0 = blockIdx.x * RPC; n0 < N; n0 += gridDim.x * RPC) {
-        int rows[RPW];
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) rows[r] = n0 + (warp / KS) * RPW + r;
+    bool have = true;  // pk holds the first step's first loads
+    for (int u0 = blockIdx.x * UPC; u0 < NU; u0 += gridDim.x * UPC) {
         float acc[RPW][BM];
 #pragma unroll
         for (int r = 0; r < RPW; ++r)
 #pragma unroll
             for (int b = 0; b < BM; ++b) acc[r][b] = 0.f;
         for (int v0 = lane; v0 < S8; v0 += 32 * kLmUnroll) {
-            uint4 pk[RPW][kLmUnroll];
-#pragma unroll
-            for (int r = 0; r < RPW; ++r) {
-                const uint4* wr = reinterpret_cast<const uint4*>(W + (long long)min(rows[r], N - 1) * K) + j0;
-#pragma unroll
-                for (int u = 0; u < kLmUnroll; ++u) {
-                    const int v8 = v0 + 32 * u;
-                    pk[r][u] = (v8 < S8 && rows[r] < N) ? __ldg(wr + v8) : make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
+            if (!have) load_w(u0, v0);
+            have = false;
 #pragma unroll
             for (int u = 0; u < kLmUnroll; ++u) {
                 const int v8 = v0 + 32 * u;
@@ -230,9 +338,7 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
                 }
             }
         }
-        // sums over the lanes (every lane ends with all of them); lane (rl, bl) = (lane /
-        // BM, lane % BM) then finishes row rl of the step for batch row bl; with KS > 1
-        // the writing warp adds the partial sums of the warps sharing its rows
+        // sums over the lanes (every lane ends with all of them)
 #pragma unroll
         for (int r = 0; r < RPW; ++r)
 #pragma unroll
@@ -241,6 +347,8 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
 #pragma unroll
                     for (int o = 16; o; o >>= 1) acc[r][b] += __shfl_xor_sync(0xffffffffu, acc[r][b], o);
                 }
+        // lane (rl, bl) = (lane / BM, lane % BM) finishes row rl of the step for batch row
+        // bl; with KS > 1 the writing warp adds the partial sums of the warps sharing its rows
         const int rl = lane / BM, bl = lane % BM;
         float a = 0.f;
 #pragma unroll
@@ -258,12 +366,24 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
             }
             __syncthreads();
         }
+        if (MIX) {
+            // lane (0, b) gathers k and v of batch row b from lanes (1, b), (2, b)
+            const float zk = __shfl_sync(0xffffffffu, a, (lane + BM) & 31);
+            const float zv = __shfl_sync(0xffffffffu, a, (lane + 2 * BM) & 31);
+            const int d = u0 + warp / KS;
+            if (mix_lane && d < NU) {
+                if (u0 != blockIdx.x * UPC)
+                    mo = lm_mixer_load(lane, d, ep.zr, ep.conv, ep.h, ep.L, B, ep.D, t, ep.Y, x);
+                lm_mixer_finish(mo, a, zk, zv, lane, d, ep.zr, ep.L, B, ep.D, t, ep.X, ep.Y, y);
+            }
+            continue;
+        }
         const bool writer = KS == 1 || warp % KS == 0;
-        const int n = n0 + (warp / KS) * RPW + rl;
+        const int n = u0 + (warp / KS) * RPW + rl;
         const bool own = writer && pair && n < N;
         if (own) {
             if (EPI == kLmGelu) a = __bfloat162float(__float2bfloat16_rn(0.5f * a * (1.0f + erff(a * 0.70710678118654752f))));
-            if (EPI == kLmAdd) y[(long long)bl * N + n] = __ldcg(y + (long long)bl * N + n) + a;
+            if (EPI == kLmAdd) y[(long long)bl * N + n] = __ldcg(ep.res + (long long)bl * N + n) + a;
             else if (EPI != kLmArgmax || y) y[(long long)bl * N + n] = a;
         }
         if (EPI == kLmArgmax) {
@@ -284,57 +404,27 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
             unsigned long long k = 0ull;
 #pragma unroll
             for (int w = 0; w < nw; ++w) k = sbest[w][threadIdx.x] > k ? sbest[w][threadIdx.x] : k;
-            if (k) atomicMax(amax + threadIdx.x, k);
+            if (k) atomicMax(ep.amax + threadIdx.x, k);
         }
     }
 }
 
-// The mixer part of layer l at token t, one thread per (b, d): short convolution of the
-// three in-projection streams (q, k, v) with the two previous tokens' values (ring
-// zr[2][B][3D], shifted here), the gate x = kc vc stored as the mixer's input at t, the
-// red cell y_t = (running sum at t) + h_0 x_t (the running sum is 0 at t = 0, where no
-// block has written), y_t kept at t, and the gated residual u += qc y_t.
-// With io (a replayed per-token graph) the token index comes from the step record.
+// The mixer step as a kernel of its own, one thread per (b, d), reading q, k, v from
+// z [B][3D] (the traced path launches it separately, so that it can be timed).  With io
+// (a replayed per-token graph) the token index comes from the step record.
 __global__ void k_lm_mixer(const float* __restrict__ z, float* __restrict__ zr, const float* __restrict__ conv,
                            const float* __restrict__ h, long long L, int B, int D, long long t, float* X,
-                           float* Y, float* u, const TokIO* io) {
+                           float* Y, const float* u, float* r, const TokIO* io) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     grid_dep_wait();
     grid_dep_launch();
     if (e >= B * D) return;
     const int b = e / D, d = e - b * D;
-    const int D3 = 3 * D;
-    // every load first (one round trip), then the arithmetic and the stores
-    float z0[3], z1[3], z2[3], c0[3], c1[3], c2[3];
-    float* r1 = zr + (long long)b * D3 + d;                      // z_{t-1}
-    float* r2 = zr + (long long)B * D3 + (long long)b * D3 + d;  // z_{t-2}
-#pragma unroll
-    for (int s = 0; s < 3; ++s) {
-        const int j = s * D + d;
-        z0[s] = __ldcg(z + b * D3 + j);
-        z1[s] = __ldcg(r1 + s * D);
-        z2[s] = __ldcg(r2 + s * D);
-        c0[s] = __ldg(conv + j);
-        c1[s] = __ldg(conv + D3 + j);
-        c2[s] = __ldg(conv + 2 * D3 + j);
-    }
-    const float h0 = __ldg(h + (long long)d * L);
-    const float u0 = __ldcg(u + e);
+    const float* zb = z + (long long)b * 3 * D + d;
+    const float zq = __ldcg(zb), zk = __ldcg(zb + D), zv = __ldcg(zb + 2 * D);
     if (io) t = io->t;
-    const long long g = (long long)b * D + d;
-    const float run = t == 0 ? 0.f : __ldcg(Y + g * L + t);
-    float zc[3];
-#pragma unroll
-    for (int s = 0; s < 3; ++s) {
-        zc[s] = fmaf(c0[s], z0[s], fmaf(c1[s], z1[s], c2[s] * z2[s]));
-        r2[s * D] = z1[s];
-        r1[s * D] = z0[s];
-    }
-    const float x = zc[1] * zc[2];
-    X[g * L + t] = x;
-    const float yv = fmaf(h0, x, run);
-    Y[g * L + t] = yv;
-    u[e] = fmaf(zc[0], yv, u0);
+    const MixOps o = lm_mixer_load(b, d, zr, conv, h, L, B, D, t, Y, u);
+    lm_mixer_finish(o, zq, zk, zv, b, d, zr, L, B, D, t, X, Y, r);
 }
 
 // next[b] = the greedy choice the LM head folded into amax[b] (largest logit, lowest id

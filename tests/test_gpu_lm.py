@@ -35,7 +35,8 @@ def margins(logits):
     return s[..., -1] - s[..., -2]
 
 
-@pytest.mark.parametrize("M,B,D,L,V,T", [(2, 2, 64, 256, 1000, 256), (3, 4, 32, 512, 300, 200)])
+@pytest.mark.parametrize("M,B,D,L,V,T", [(2, 2, 64, 256, 1000, 256), (3, 4, 32, 512, 300, 200),
+                                          (2, 6, 40, 128, 700, 128)])
 def test_teacher_forced_logits_and_choices_match_oracle(M, B, D, L, V, T):
     p = synth.hyena_params(M, D, L, V, seed=1)
     tok = synth.token_ids(T, B, V, seed=2)
@@ -120,3 +121,23 @@ def test_generation_from_graphs_equals_host_launches():
             outs.append(nxt)
     np.testing.assert_array_equal(outs[0], outs[1])
     np.testing.assert_array_equal(outs[0], outs[2])
+
+
+def test_traced_run_with_its_own_mixer_kernel_equals_the_fused_run():
+    # a traced run launches the mixer step as its own kernel after a plain in-projection;
+    # otherwise it is fused into the in-projection's epilogue: the same fp32 operations,
+    # so the same choices and logits, bit for bit
+    M, B, D, L, V = 2, 4, 64, 256, 500
+    p = synth.hyena_params(M, D, L, V, seed=13)
+    tok = synth.token_ids(L, B, V, seed=14)
+    outs = []
+    with model(p, M, B, D, L, V) as lm:
+        for trace in (False, True):
+            lm.reset()
+            lm.set_trace(trace)
+            logits = np.empty((64, B, V), np.float32)
+            nxt = np.empty((64, B), np.int32)
+            lm.forward(tok[:64], 64, logits, nxt)
+            outs.append((logits, nxt))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
