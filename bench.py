@@ -234,6 +234,8 @@ def main():
     ap.add_argument("--lm", action="store_true",
                     help="the Hyena-like language model end to end (18 layers, B=4, D=768, L=2^15, vocabulary "
                          "50257, greedy decoding): tokens/s and the mixer / non-mixer split")
+    ap.add_argument("--lm-profile", type=int, default=0, metavar="N",
+                    help="with --lm: generate the first N tokens from host launches, untimed (for ncu launch lists)")
     ap.add_argument("--prefill", default=None,
                     help="comma-separated prompt lengths: time fi_prefill against the online "
                          "teacher-forced path over the same prompt (headline stack)")
@@ -712,6 +714,16 @@ def bench_lm(args):
     lm = fi.LanguageModel(M, B, D, L, V, p["E"], p["W_lm"], stack("W_in"), stack("c"), stack("W1"), stack("W2"),
                           stack("h"))
     tok0_d = torch.from_numpy(tok0).cuda()
+    if args.lm_profile:
+        # a profiling workload, not a measurement: one generation of the first
+        # lm_profile tokens, every kernel launched from the host (for ncu launch lists)
+        lm.set_graphs(False)
+        out = torch.empty((args.lm_profile, B), dtype=torch.int32, device="cuda")
+        lm.generate(tok0_d, args.lm_profile, out)
+        torch.cuda.synchronize()
+        lm.close()
+        print(json.dumps({"lm_profile_tokens": args.lm_profile, "last_choices": out[-1].tolist()}), flush=True)
+        return 0
     nxt = torch.empty((L, B), dtype=torch.int32, device="cuda")
 
     def gen():
