@@ -309,6 +309,48 @@ int fi_lm_set_trace(fi_lm *m, int on);
  * every token).  Synchronises. */
 int fi_lm_split(fi_lm *m, double *mixer_us, double *total_us);
 
+/* ---------------------------------------------------------------- data-dependent filter
+ * The long convolution with a filter that depends on the data (the Flash Inference
+ * summary, section "Technische Innovationen" item 4, "Datenabhaengige
+ * Filter-Erweiterung"; the rebuttal's answer on data-dependent filters: a different
+ * tiling with two FFT convolutions of the same size per step, at twice the cost).  G
+ * independent channels; at step t the input x_t and the filter value rho_t of every
+ * channel arrive together, and
+ *     y_t = sum_{i + j = t} rho_i x_j
+ * is returned before step t + 1 (the definition is the causal convolution; only what
+ * is known when differs from a fixed filter).  Tiling (the appendix that holds the
+ * pages' algorithm is not on the pages; this is the reading the library follows):
+ * red cells rho_0 x_t + rho_t x_0 at step t; after the n-th token, U = lowbit(n),
+ * Algorithm 1's block with x[n-U, n) as the input and rho[0, 2U) as the taps and,
+ * unless n is a power of two, the same block with the roles swapped; at n = U the
+ * x-block runs while rho[U, 2U) is still zero, which adds exactly the products of the
+ * first U values of both sequences that are still due.  A block of size U takes the
+ * direct tau or the FFT tau against the spectra of the prefixes x[0, 2U), rho[0, 2U),
+ * made once at step 2U (when they are final; first used at step 3U).
+ * Layout: x, rho and the running sums are [G][L] float32 on the device. */
+typedef struct fi_dd fi_dd;
+
+/* G >= 1 channels; L a power of two, 2 <= L <= 2^17.  Device memory: 3 G L floats plus
+ * about 2.5 G L complex values of spectra.  Returns NULL on error (fi_last_error). */
+fi_dd *fi_dd_create(int G, int L);
+
+/* Release the context.  NULL is accepted. */
+void fi_dd_destroy(fi_dd *d);
+
+/* Back to step 0 (clears the buffers). */
+int fi_dd_reset(fi_dd *d);
+
+/* Steps t .. t+steps-1: x and rho [steps][G] float32 (host or device) are the inputs of
+ * those steps; y [steps][G] (host or device) receives the outputs.  FI_ECAPACITY past
+ * L; FI_EINVAL for a NULL array with steps > 0. */
+int fi_dd_forward(fi_dd *d, const float *x, const float *rho, int steps, float *y);
+
+/* The implementation of blocks of size 2^q: FI_TAU_DIRECT (q <= 12), FI_TAU_FFT
+ * (q >= 3), or FI_TAU_AUTO for the default (direct up to U = 16, FFT above).  Only
+ * before step 1 (FI_ESTATE after): the FFT form needs the prefix spectra made at
+ * step 2U. */
+int fi_dd_set_tau(fi_dd *d, int q, int impl);
+
 /* Message of the last failure on the calling thread ("" if none). */
 const char *fi_last_error(void);
 

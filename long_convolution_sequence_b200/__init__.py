@@ -73,6 +73,11 @@ SIGNATURES = {
     "fi_lm_set_trace": (_I, [_P, _I]),
     "fi_lm_set_graphs": (_I, [_P, _I]),
     "fi_lm_split": (_I, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
+    "fi_dd_create": (_P, [_I, _I]),
+    "fi_dd_destroy": (None, [_P]),
+    "fi_dd_reset": (_I, [_P]),
+    "fi_dd_forward": (_I, [_P, _P, _P, _I, _P]),
+    "fi_dd_set_tau": (_I, [_P, _I, _I]),
     "fi_last_error": (ctypes.c_char_p, []),
     "fi_version": (ctypes.c_char_p, []),
 }
@@ -284,6 +289,43 @@ class LanguageModel:
         a, b = ctypes.c_double(), ctypes.c_double()
         _check(get_lib().fi_lm_split(self._h, ctypes.byref(a), ctypes.byref(b)))
         return a.value, b.value
+
+
+class DataDependentConvolution:
+    """The long convolution with a filter that arrives online with the data
+    (fi_dd_create .. fi_dd_destroy): G channels, y_t = sum_{i+j=t} rho_i x_j, both x_t
+    and rho_t given at step t.  Arrays are float32 [steps][G], host or device."""
+
+    def __init__(self, G: int, L: int):
+        self.G, self.L = G, L
+        lib = get_lib()
+        h = lib.fi_dd_create(G, L)
+        if not h:
+            raise FiError(FI_EINVAL, last_error())
+        self._h = h
+        self._lib = lib
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.fi_dd_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def reset(self):
+        _check(get_lib().fi_dd_reset(self._h))
+
+    def set_tau(self, q: int, impl: int):
+        _check(get_lib().fi_dd_set_tau(self._h, q, impl))
+
+    def forward(self, x, rho, steps, y):
+        _check(get_lib().fi_dd_forward(self._h, _ptr(x), _ptr(rho), steps, _ptr(y)))
 
 
 def tau(impl: int, U: int, blocks, taps, out, accumulate: bool = False):

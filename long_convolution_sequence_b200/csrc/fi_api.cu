@@ -27,6 +27,7 @@
 #include "fi.h"
 #include "fi_kernels.cuh"
 #include "fi_lm.cuh"
+#include "fi_dd.cuh"
 
 using namespace fi;
 
@@ -2109,6 +2110,260 @@ int fi_lm_split(fi_lm* m, double* mixer_us, double* total_us) {
     }
     const double scale = m->sampled_tokens ? (double)m->traced_tokens / (double)m->sampled_tokens : 0.0;
     *mixer_us = blocks + steps * scale;
+    return FI_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- data-dependent filter
+// The long convolution with a filter that arrives online with the data (fi.h,
+// fi_dd_create): red cells per step (k_dd_red), then the blocks released after the
+// step's token: two of the same size U = lowbit(n) at a step n that is not a power of
+// two (x against rho's prefix, rho against x's prefix), one at n = U (x against rho
+// with its unknown tail still zero).  The FFT form uses the spectra of the prefixes
+// x[0, 2U) and rho[0, 2U), made at step 2U; the power-of-two block uses the spectrum
+// of rho[0, 2U) made at its own step.
+
+constexpr unsigned kDdMagic = 0xDD5EED01u;
+
+struct fi_dd {
+    unsigned magic = kDdMagic;
+    fi_ctx* c = nullptr;                 // device, stream, twiddles, allocation count
+    int G = 0, L = 0, P = 0;
+    long long t = 0;
+    float *xb = nullptr, *rb = nullptr;  // [G][L]: x and rho as they arrive (zero beyond t)
+    float* acc = nullptr;                // [G][L]: running sums of the products i, j >= 1
+    float2* spx[32] = {};                // per q: spectra of x[0, 2^(q+1)), stride 2^q + 2
+    float2* spr[32] = {};                // per q: spectra of rho[0, 2^(q+1))
+    float2* spz = nullptr;               // spectra of rho[0, 2U) at the power-of-two step U
+    int tau_user[32] = {};
+    float* stage = nullptr;              // host arrays staged on the device
+    size_t stage_n = 0;
+};
+
+namespace {
+
+std::mutex g_dd_mu;
+std::set<const fi_dd*> g_dd_live;
+
+int check_dd(const fi_dd* d) {
+    std::lock_guard<std::mutex> lk(g_dd_mu);
+    if (!d || !g_dd_live.count(d) || d->magic != kDdMagic) return set_err(FI_ESTATE, "null or destroyed context");
+    return FI_OK;
+}
+
+// Blocks of size 2^q: the direct tau up to U = 8 (one thread per tile), the FFT tau
+// above, unless set otherwise.
+int dd_tau(const fi_dd* d, int q) {
+    if (d->tau_user[q]) return d->tau_user[q];
+    return q <= 3 ? FI_TAU_DIRECT : FI_TAU_FFT;
+}
+
+// Algorithm 1's block released after the n-th token over all channels: input x (or
+// rho) at [n - U, n), taps rho (or x) from index 0, added onto the running sums.
+int dd_block(fi_dd* d, long long n, bool x_input, const float2* spec, cudaStream_t st) {
+    TileArgs a;
+    memset(&a, 0, sizeof(a));
+    a.act = x_input ? d->xb : d->rb;
+    a.act_out = d->acc;
+    a.h = x_input ? d->rb : d->xb;
+    a.L = d->L;
+    a.G = d->G;
+    a.D = d->G;
+    a.n = n;
+    a.U = (int)lowbit(n);
+    a.count = d->G;
+    a.overwrite = 0;
+    a.tw = d->c->tw;
+    a.twlog = kTwLog;
+    const int q = ctz64(n);
+    if (dd_tau(d, q) == FI_TAU_DIRECT) return launch_direct_tile(a, st);
+    a.spec = spec;
+    a.spec_stride = fused_stride(a.U);
+    return launch_fft(q, a, st);
+}
+
+int dd_run(fi_dd* d, const float* x, const float* rho, int steps, float* y, cudaStream_t st) {
+    const int G = d->G;
+    const long long L = d->L;
+    int rc;
+    for (int k = 0; k < steps; ++k) {
+        const long long t = d->t + k;
+        k_dd_red<<<(G + 255) / 256, 256, 0, st>>>(d->xb, d->rb, d->acc, x + (size_t)k * G, rho + (size_t)k * G,
+                                                  y + (size_t)k * G, t, G, L);
+        CK(cudaGetLastError());
+        const long long n = t + 1;
+        if (n >= L) continue;
+        const int q = ctz64(n);
+        if (is_pow2(n)) {
+            // the prefixes of length n are final: spectra for the blocks of size n / 2
+            // still to come (steps 3n/2, 5n/2, ...)
+            if (q >= 1) {
+                const int q2 = q - 1;
+                if (dd_tau(d, q2) == FI_TAU_FFT && (3LL << q2) < L) {
+                    if ((rc = make_spectra(q2, d->xb, L, G, d->spx[q2], d->c->tw, st))) return rc;
+                    if ((rc = make_spectra(q2, d->rb, L, G, d->spr[q2], d->c->tw, st))) return rc;
+                }
+            }
+            if (dd_tau(d, q) == FI_TAU_FFT && (rc = make_spectra(q, d->rb, L, G, d->spz, d->c->tw, st))) return rc;
+            if ((rc = dd_block(d, n, true, d->spz, st))) return rc;
+        } else {
+            if ((rc = dd_block(d, n, true, d->spr[q], st))) return rc;
+            if ((rc = dd_block(d, n, false, d->spx[q], st))) return rc;
+        }
+    }
+    return FI_OK;
+}
+
+void dd_free(fi_dd* d) {
+    if (!d) return;
+    if (d->c) cudaStreamSynchronize(d->c->stream);
+    cudaFree(d->xb);
+    cudaFree(d->rb);
+    cudaFree(d->acc);
+    for (int q = 0; q < 32; ++q) {
+        cudaFree(d->spx[q]);
+        cudaFree(d->spr[q]);
+    }
+    cudaFree(d->spz);
+    cudaFree(d->stage);
+    free_ctx(d->c);
+    d->magic = 0;
+    delete d;
+}
+
+int dd_create_impl(fi_dd* d) {
+    int rc = set_all_attrs();
+    if (rc) return rc;
+    fi_ctx* c = new fi_ctx();
+    d->c = c;
+    CK(cudaGetDevice(&c->dev));
+    CK(cudaDeviceGetAttribute(&c->nsm, cudaDevAttrMultiProcessorCount, c->dev));
+    if ((rc = upload_twiddles(c))) return rc;
+    const size_t GL = (size_t)d->G * d->L;
+    if ((rc = dev_alloc(c, &d->xb, GL)) || (rc = dev_alloc(c, &d->rb, GL)) || (rc = dev_alloc(c, &d->acc, GL)))
+        return rc;
+    // prefix spectra for every size of the blocks at steps that are not powers of two
+    // (3U < L), the power-of-two block's spectrum for U up to L / 2
+    for (int q = kFftQMin; q <= d->P - 2; ++q) {
+        const size_t n = (size_t)d->G * fused_stride(1LL << q);
+        if ((rc = dev_alloc(c, &d->spx[q], n)) || (rc = dev_alloc(c, &d->spr[q], n))) return rc;
+    }
+    if (d->P - 1 >= kFftQMin && (rc = dev_alloc(c, &d->spz, (size_t)d->G * fused_stride(1LL << (d->P - 1)))))
+        return rc;
+    CK(cudaMemset(d->xb, 0, GL * sizeof(float)));
+    CK(cudaMemset(d->rb, 0, GL * sizeof(float)));
+    CK(cudaMemset(d->acc, 0, GL * sizeof(float)));
+    CK(cudaDeviceSynchronize());
+    return FI_OK;
+}
+
+// A host array of n floats on the device (device arrays pass through).
+int dd_stage(fi_dd* d, const float* src, size_t n, size_t off, const float** out, cudaStream_t st) {
+    if (is_device_ptr(src)) {
+        *out = src;
+        return FI_OK;
+    }
+    CK(cudaMemcpyAsync(d->stage + off, src, n * sizeof(float), cudaMemcpyHostToDevice, st));
+    *out = d->stage + off;
+    return FI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fi_dd* fi_dd_create(int G, int L) {
+    g_err[0] = 0;
+    if (G < 1 || L < 2 || (L & (L - 1)) || L > (1 << kFftQMax)) {
+        set_err(FI_EINVAL, "fi_dd_create: need G >= 1 and L a power of two in [2, %d] (G=%d, L=%d)",
+                1 << kFftQMax, G, L);
+        return nullptr;
+    }
+    fi_dd* d = new fi_dd();
+    d->G = G;
+    d->L = L;
+    while ((1 << d->P) < L) ++d->P;
+    const int rc = dd_create_impl(d);
+    if (rc) {
+        const std::string msg = g_err;
+        dd_free(d);
+        cudaGetLastError();
+        set_err(rc, "%s", msg.c_str());
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_dd_mu);
+    g_dd_live.insert(d);
+    return d;
+}
+
+void fi_dd_destroy(fi_dd* d) {
+    {
+        std::lock_guard<std::mutex> lk(g_dd_mu);
+        if (!d || !g_dd_live.count(d)) return;
+        g_dd_live.erase(d);
+    }
+    dd_free(d);
+}
+
+int fi_dd_reset(fi_dd* d) {
+    int rc = check_dd(d);
+    if (rc) return rc;
+    const size_t GL = (size_t)d->G * d->L;
+    cudaStream_t st = d->c->stream;
+    CK(cudaMemsetAsync(d->xb, 0, GL * sizeof(float), st));
+    CK(cudaMemsetAsync(d->rb, 0, GL * sizeof(float), st));
+    CK(cudaMemsetAsync(d->acc, 0, GL * sizeof(float), st));
+    CK(cudaStreamSynchronize(st));
+    d->t = 0;
+    return FI_OK;
+}
+
+int fi_dd_set_tau(fi_dd* d, int q, int impl) {
+    int rc = check_dd(d);
+    if (rc) return rc;
+    if (q < 0 || q >= d->P) return set_err(FI_EINVAL, "fi_dd_set_tau: q=%d outside [0, %d)", q, d->P);
+    if (impl != FI_TAU_AUTO && impl != FI_TAU_DIRECT && impl != FI_TAU_FFT)
+        return set_err(FI_EINVAL, "fi_dd_set_tau: unknown implementation %d", impl);
+    if (impl == FI_TAU_DIRECT && q > kDirectQMax)
+        return set_err(FI_EINVAL, "fi_dd_set_tau: the direct tau serves U <= %d", 1 << kDirectQMax);
+    if (impl == FI_TAU_FFT && q < kFftQMin)
+        return set_err(FI_EINVAL, "fi_dd_set_tau: the FFT tau serves U >= %d", 1 << kFftQMin);
+    if (d->t > 0) return set_err(FI_ESTATE, "fi_dd_set_tau: only before the first step (t=%lld)", d->t);
+    d->tau_user[q] = impl;
+    return FI_OK;
+}
+
+int fi_dd_forward(fi_dd* d, const float* x, const float* rho, int steps, float* y) {
+    int rc = check_dd(d);
+    if (rc) return rc;
+    if (steps < 0) return set_err(FI_EINVAL, "steps must be >= 0");
+    if (d->t + steps > d->L)
+        return set_err(FI_ECAPACITY, "t=%lld + steps=%d exceeds capacity L=%d", d->t, steps, d->L);
+    if (steps == 0) return FI_OK;
+    if (!x || !rho || !y) return set_err(FI_EINVAL, "fi_dd_forward: NULL array");
+    const size_t n = (size_t)steps * d->G;
+    const bool xh = !is_device_ptr(x), rh = !is_device_ptr(rho), yh = !is_device_ptr(y);
+    const size_t need = n * ((xh ? 1 : 0) + (rh ? 1 : 0) + (yh ? 1 : 0));
+    if (need > d->stage_n) {
+        cudaFree(d->stage);
+        d->stage = nullptr;
+        d->stage_n = 0;
+        if ((rc = dev_alloc(d->c, &d->stage, need))) return rc;
+        d->stage_n = need;
+    }
+    cudaStream_t st = d->c->stream;
+    size_t off = 0;
+    const float *xd = nullptr, *rd = nullptr;
+    if ((rc = dd_stage(d, x, n, off, &xd, st))) return rc;
+    off += xh ? n : 0;
+    if ((rc = dd_stage(d, rho, n, off, &rd, st))) return rc;
+    off += rh ? n : 0;
+    float* yd = yh ? d->stage + off : y;
+    if ((rc = dd_run(d, xd, rd, steps, yd, st))) return rc;
+    d->t += steps;
+    if (yh) CK(cudaMemcpyAsync(y, yd, n * sizeof(float), cudaMemcpyDeviceToHost, st));
+    CK(cudaStreamSynchronize(st));
     return FI_OK;
 }
 

@@ -15,8 +15,9 @@ paper summary, section "Experimentelle Einrichtung"):
   ``x_0 ~ N(0,1)`` per (b, c).
 
 Generator: numpy PCG64 seeded through ``SeedSequence([seed, stream, l])``, one
-independent stream per layer (stream 1), one for teacher-forced inputs (stream 2)
-and one for the closed-loop start token (stream 3).  Within a layer stream the
+independent stream per layer (stream 1), one for teacher-forced inputs (stream 2),
+one for the closed-loop start token (stream 3), the Hyena-like model's weights
+(stream 4), its token ids (stream 5) and the data-dependent filter's inputs (stream 6).  Within a layer stream the
 draw order is: ``a_c`` for all c, then the normals in [c][k] order.
 """
 from __future__ import annotations
@@ -160,6 +161,36 @@ def hyena_params(M: int, D: int, L: int, V: int, seed: int = 0) -> dict:
 def token_ids(T: int, B: int, V: int, seed: int = 0) -> np.ndarray:
     """int32 [T][B] synthetic token ids, uniform over the vocabulary (stream 5)."""
     return _rng(seed, 5).integers(0, V, size=(T, B)).astype(np.int32)
+
+
+def dd_inputs(T: int, G: int, seed: int = 0):
+    """The data-dependent filter's online inputs (stream 6): x [T][G] ~ N(0, 1) and
+    rho [T][G] with the filter law of ``filters`` laid out by step, rho[t][g] =
+    N(0, 1) * exp(-a_g t) / sqrt(32), a_g ~ U(0.001, 0.05) (a_g drawn first, then the
+    normals of x, then those of rho, [t][g] order).  float32."""
+    g = _rng(seed, 6)
+    a = g.uniform(A_LO, A_HI, size=G)
+    x = g.standard_normal((T, G)).astype(np.float32)
+    z = g.standard_normal((T, G))
+    rho = (z * np.exp(-np.outer(np.arange(T, dtype=np.float64), a)) * SCALE).astype(np.float32)
+    return x, rho
+
+
+def device_dd_inputs(T: int, G: int, seed: int = 0):
+    """``dd_inputs``' law drawn on the device by torch's seeded CUDA generator
+    (``manual_seed(1000003 * seed + 6)``: a, then x, then the normals of rho): a
+    different draw, for sizes whose host generation would take minutes.  Torch CUDA
+    tensors [T][G]."""
+    import torch
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1_000_003 * seed + 6)
+    a = torch.empty(G, device="cuda").uniform_(A_LO, A_HI, generator=gen)
+    x = torch.empty((T, G), device="cuda").normal_(generator=gen)
+    rho = torch.empty((T, G), device="cuda").normal_(generator=gen)
+    t = torch.arange(T, device="cuda", dtype=torch.float32)
+    for t0 in range(0, T, 4096):
+        rho[t0:t0 + 4096] *= torch.exp(-t[t0:t0 + 4096, None] * a[None, :]) * SCALE
+    return x, rho
 
 
 # Workloads (layers, B, D, L) of the measured configurations.
