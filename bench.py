@@ -239,7 +239,12 @@ def main():
     ap.add_argument("--prefill", default=None,
                     help="comma-separated prompt lengths: time fi_prefill against the online "
                          "teacher-forced path over the same prompt (headline stack)")
+    ap.add_argument("--dd", action="store_true",
+                    help="the long convolution with a data-dependent filter (18 x 864 channels, L=2^17, "
+                         "both sequences online): channel-steps/s, against a fixed filter of the same shape")
     args = ap.parse_args()
+    if args.dd:
+        return bench_dd(args)
     if args.prefill:
         return bench_prefill(args)
     if args.sweep:
@@ -795,6 +800,118 @@ def bench_lm(args):
             "clocks": clk, "setup_s": {"params": round(t_gen, 1)}}
     print(json.dumps(line), flush=True)
     return 0
+
+DD_CONFIG = dict(G=18 * 864, L=1 << 17)
+
+
+def dd_model_bytes(G, L):
+    """Algorithmic bytes of one online pass of the data-dependent convolution: per
+    channel, every block of size U moves 4U(3B+2) = 20U bytes at B = 1 (its U inputs,
+    its taps' 2U values or their spectrum, U outputs read and written), two blocks at
+    every step that is not a power of two; the red cell reads the running sum, x_0 and
+    rho_0 and writes x_t, rho_t, y_t (24 bytes)."""
+    total = 0
+    for n in range(1, L):
+        U = n & -n
+        total += 20 * U * (1 if (n & (n - 1)) == 0 else 2)
+    return G * (total + 24 * L)
+
+
+def bench_dd(args):
+    """The long convolution with a data-dependent filter (the pages' extension with
+    two convolutions of the same size per step): one online pass of L steps over G
+    channels, both sequences drawn on the device (synth.device_dd_inputs), every
+    launch from the host, CUDA events around each pass.  Beside it the same shape with
+    the filter fixed (rho of this draw as a precomputed filter) through Algorithm 1 on
+    the per-token path with host launches: their ratio is the pages' factor of two.
+    The oracle (fp64 causal convolution) on a bounded sample of channels and steps."""
+    import torch
+    import long_convolution_sequence_b200 as fi
+    from long_convolution_sequence_b200 import synth
+    G, L = DD_CONFIG["G"], DD_CONFIG["L"]
+    x, rho = synth.device_dd_inputs(L, G, seed=0)
+    y = torch.empty((L, G), device="cuda")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dd = fi.DataDependentConvolution(G, L)
+    for _ in range(max(1, min(args.warmup, 1))):
+        dd.reset()
+        dd.forward(x, rho, L, y)
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 2))
+    clocks = Clocks(0)
+    clocks.start()
+    ms = []
+    for _ in range(steps):
+        dd.reset()
+        ev0.record()
+        dd.forward(x, rho, L, y)
+        ev1.record()
+        torch.cuda.synchronize()
+        ms.append(ev0.elapsed_time(ev1))
+    clk = clocks.stop()
+    t_dd = min(ms)
+    # sampled parity of the timed pass: 4 channels over the first 4096 steps
+    import oracle
+    chans = [0, 1, G // 2, G - 1]
+    Ts = 4096
+    xs = x[:Ts, chans].cpu().numpy()
+    rs = rho[:Ts, chans].cpu().numpy()
+    ref = oracle.causal_conv_batch(np.ascontiguousarray(rs.T), np.ascontiguousarray(xs.T)).T
+    got = y[:Ts, chans].cpu().numpy()
+    err = float(np.abs(got - ref).max() / np.sqrt(np.mean(ref ** 2)))
+    dd.close()
+    del y
+    torch.cuda.empty_cache()
+    # the fixed filter of the same shape: one layer of G channels, filter = this rho
+    h = rho.t().contiguous().view(1, G, L)
+    ctx = fi.FlashInference(1, 1, G, L, h)
+    del h
+    torch.cuda.empty_cache()
+    ctx.set_path(fi.FI_PATH_TOKEN)
+    ctx.set_graphs(False)
+    yy = torch.empty((L, 1, G), device="cuda")
+    xv = x.view(L, 1, G)
+    ctx.reset()
+    ctx.forward(xv, L, yy)
+    torch.cuda.synchronize()
+    ctx.reset()
+    ev0.record()
+    ctx.forward(xv, L, yy)
+    ev1.record()
+    torch.cuda.synchronize()
+    t_fixed = ev0.elapsed_time(ev1)
+    ctx.close()
+    # CPU oracle on a bounded sample: the lazy causal convolution of 16 channels over
+    # the first T_s steps, scaled to G channels and L steps by the lazy cost T (T+1) / 2
+    T_s = 1 << 14
+    xc = x[:T_s, :16].cpu().numpy()
+    rc = rho[:T_s, :16].cpu().numpy()
+    t0 = time.perf_counter()
+    oracle.causal_conv_batch(np.ascontiguousarray(rc.T), np.ascontiguousarray(xc.T))
+    sec = time.perf_counter() - t0
+    scale = (G / 16.0) * (L * (L + 1) / 2.0) / (T_s * (T_s + 1) / 2.0)
+    hbm, src, _ = peaks()
+    nbytes = dd_model_bytes(G, L)
+    ach = nbytes / (t_dd / 1e3) / 1e9
+    line = {"metric": "data-dependent filter: channel-steps/s (G*L/time), both sequences online",
+            "value": round(G * L / (t_dd / 1e3), 1), "unit": "channel-steps/s", "ms_per_pass": round(t_dd, 2),
+            "steps": steps, "higher_is_better": True, "dtype": "f32",
+            "data": "synthetic: x ~ N(0,1), rho with the filters' law laid out by step (drawn on the device)",
+            "config": {"workload": "data-dependent filter, %d channels (18 x 864), L=%d" % (G, L), "G": G, "L": L,
+                       "launches": "host, per step: red cells + 1 or 2 blocks (+ prefix spectra at powers of two)"},
+            "fixed_filter": {"ms_per_pass": round(t_fixed, 2), "path": "Algorithm 1, per-token path, host launches",
+                             "ratio_dd_over_fixed": round(t_dd / t_fixed, 3)},
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(ach / hbm, 4), "traffic": None, "kernel": "whole pass",
+                         "model_bytes": nbytes, "peak_source": src + " (MEASURED_PEAKS.json hbm_gbs)"},
+            "parity_sample": {"channels": chans, "steps": Ts, "max_err_over_rms": err},
+            "cpu_baseline": {"value": round(G * L / (sec * scale), 3), "unit": "channel-steps/s", "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": "16 channels x first %d steps, lazy fp64, scaled by channels and T(T+1)/2" % T_s},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
 
 def bench_prefill(args):
     """Prompt prefill (fi_prefill: one FFT convolution per layer) against the online

@@ -346,9 +346,9 @@ int fi_dd_reset(fi_dd *d);
 int fi_dd_forward(fi_dd *d, const float *x, const float *rho, int steps, float *y);
 
 /* The implementation of blocks of size 2^q: FI_TAU_DIRECT (q <= 12), FI_TAU_FFT
- * (q >= 3), or FI_TAU_AUTO for the default (direct up to U = 16, FFT above).  Only
- * before step 1 (FI_ESTATE after): the FFT form needs the prefix spectra made at
- * step 2U. */
+ * (q >= 3), or FI_TAU_AUTO for the default (direct up to U = 8, added by the step
+ * kernel itself; FFT above).  Only before step 1 (FI_ESTATE after): the FFT form needs
+ * the prefix spectra made at step 2U. */
 int fi_dd_set_tau(fi_dd *d, int q, int impl);
 
 /* Message of the last failure on the calling thread ("" if none). */

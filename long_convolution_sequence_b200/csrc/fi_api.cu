@@ -2117,8 +2117,8 @@ int fi_lm_split(fi_lm* m, double* mixer_us, double* total_us) {
 
 // ---------------------------------------------------------------- data-dependent filter
 // The long convolution with a filter that arrives online with the data (fi.h,
-// fi_dd_create): red cells per step (k_dd_red), then the blocks released after the
-// step's token: two of the same size U = lowbit(n) at a step n that is not a power of
+// fi_dd_create): red cells per step (k_dd_step, which also adds the blocks of U <= 8
+// on the direct tau), then the larger blocks released after the step's token: two of the same size U = lowbit(n) at a step n that is not a power of
 // two (x against rho's prefix, rho against x's prefix), one at n = U (x against rho
 // with its unknown tail still zero).  The FFT form uses the spectra of the prefixes
 // x[0, 2U) and rho[0, 2U), made at step 2U; the power-of-two block uses the spectrum
@@ -2189,12 +2189,22 @@ int dd_run(fi_dd* d, const float* x, const float* rho, int steps, float* y, cuda
     int rc;
     for (int k = 0; k < steps; ++k) {
         const long long t = d->t + k;
-        k_dd_red<<<(G + 255) / 256, 256, 0, st>>>(d->xb, d->rb, d->acc, x + (size_t)k * G, rho + (size_t)k * G,
-                                                  y + (size_t)k * G, t, G, L);
-        CK(cudaGetLastError());
         const long long n = t + 1;
-        if (n >= L) continue;
-        const int q = ctz64(n);
+        const int q = n < L ? ctz64(n) : -1;
+        // blocks of U <= 8 on the direct tau run inside the step kernel
+        const int fused = (q >= 0 && q <= 3 && dd_tau(d, q) == FI_TAU_DIRECT) ? (1 << q) : 0;
+        const dim3 grid((G + 255) / 256), blk(256);
+        const float *xk = x + (size_t)k * G, *rk = rho + (size_t)k * G;
+        float* yk = y + (size_t)k * G;
+        switch (fused) {
+            case 1: k_dd_step<1><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
+            case 2: k_dd_step<2><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
+            case 4: k_dd_step<4><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
+            case 8: k_dd_step<8><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
+            default: k_dd_step<0><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
+        }
+        CK(cudaGetLastError());
+        if (n >= L || fused) continue;
         if (is_pow2(n)) {
             // the prefixes of length n are final: spectra for the blocks of size n / 2
             // still to come (steps 3n/2, 5n/2, ...)

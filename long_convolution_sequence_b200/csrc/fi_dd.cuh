@@ -16,10 +16,16 @@ namespace fi {
 // Step t for every channel g: x_t and rho_t join the buffers (x, rho [G][L]), and
 // y_t = (running sum at t) + rho_0 x_t + rho_t x_0  (t > 0),  rho_0 x_0  (t = 0).
 // The running sum holds every product rho_i x_j with i, j >= 1 and i + j = t, added by
-// the blocks released after tokens 1 .. t.
-__global__ void k_dd_red(float* __restrict__ xb, float* __restrict__ rb, const float* __restrict__ acc,
-                         const float* __restrict__ x_t, const float* __restrict__ rho_t, float* __restrict__ y_t,
-                         long long t, int G, long long L) {
+// the blocks released after tokens 1 .. t.  With U > 0 the same thread then adds the
+// blocks of size U released after token n = t + 1 (U = lowbit(n) <= 8, the direct
+// tau): x[n - U, n) against rho[0, 2U) and, unless n is a power of two, rho[n - U, n)
+// against x[0, 2U), onto the running sums [n, n + U) of its channel.  Its reads are
+// its own channel's values, written by earlier steps or just now by this thread; at a
+// power of two rho[U, 2U) is still zero, as the tiling needs.
+template <int U>
+__global__ void k_dd_step(float* __restrict__ xb, float* __restrict__ rb, float* __restrict__ acc,
+                          const float* __restrict__ x_t, const float* __restrict__ rho_t, float* __restrict__ y_t,
+                          long long t, int G, long long L) {
     const int g = blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= G) return;
     const long long row = (long long)g * L;
@@ -34,6 +40,31 @@ __global__ void k_dd_red(float* __restrict__ xb, float* __restrict__ rb, const f
     xb[row + t] = xv;
     rb[row + t] = rv;
     y_t[g] = y;
+    if (U > 0) {
+        const long long n = t + 1;
+        const bool both = (n & (n - 1)) != 0;
+        float xi[U > 0 ? U : 1], ri[U > 0 ? U : 1], xp[U > 0 ? 2 * U : 1], rp[U > 0 ? 2 * U : 1];
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            xi[j] = xb[row + n - U + j];
+            ri[j] = rb[row + n - U + j];
+        }
+#pragma unroll
+        for (int k = 1; k < 2 * U; ++k) {
+            xp[k] = xb[row + k];
+            rp[k] = rb[row + k];
+        }
+#pragma unroll
+        for (int r = 0; r < U; ++r) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                s = fmaf(xi[j], rp[U + r - j], s);
+                if (both) s = fmaf(ri[j], xp[U + r - j], s);
+            }
+            acc[row + n + r] += s;
+        }
+    }
 }
 
 }  // namespace fi
