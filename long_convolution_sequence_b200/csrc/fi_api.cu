@@ -2193,7 +2193,7 @@ int dd_run(fi_dd* d, const float* x, const float* rho, int steps, float* y, cuda
         const int q = n < L ? ctz64(n) : -1;
         // blocks of U <= 8 on the direct tau run inside the step kernel
         const int fused = (q >= 0 && q <= 3 && dd_tau(d, q) == FI_TAU_DIRECT) ? (1 << q) : 0;
-        const dim3 grid((G + 255) / 256), blk(256);
+        const dim3 grid((G + 127) / 128), blk(128);
         const float *xk = x + (size_t)k * G, *rk = rho + (size_t)k * G;
         float* yk = y + (size_t)k * G;
         switch (fused) {

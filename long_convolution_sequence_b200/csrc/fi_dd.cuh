@@ -29,31 +29,36 @@ __global__ void k_dd_step(float* __restrict__ xb, float* __restrict__ rb, float*
     const int g = blockIdx.x * blockDim.x + threadIdx.x;
     if (g >= G) return;
     const long long row = (long long)g * L;
+    const long long n = t + 1;
+    // every load first, in one round trip: this step's values, the prefixes' first
+    // values, the running sum at t and, with a block, its inputs, taps and outputs
+    // (the value at position t is this step's own, taken from registers)
     const float xv = x_t[g], rv = rho_t[g];
-    float y;
-    if (t == 0) {
-        y = rv * xv;
-    } else {
-        const float x0 = xb[row], r0 = rb[row], run = acc[row + t];
-        y = fmaf(r0, xv, fmaf(rv, x0, run));
-    }
-    xb[row + t] = xv;
-    rb[row + t] = rv;
-    y_t[g] = y;
+    const float x0 = t == 0 ? xv : xb[row], r0 = t == 0 ? rv : rb[row];
+    const float run = t == 0 ? 0.f : acc[row + t];
+    constexpr int UU = U > 0 ? U : 1;
+    float xi[UU], ri[UU], xp[2 * UU], rp[2 * UU], ao[UU];
     if (U > 0) {
-        const long long n = t + 1;
-        const bool both = (n & (n - 1)) != 0;
-        float xi[U > 0 ? U : 1], ri[U > 0 ? U : 1], xp[U > 0 ? 2 * U : 1], rp[U > 0 ? 2 * U : 1];
 #pragma unroll
         for (int j = 0; j < U; ++j) {
-            xi[j] = xb[row + n - U + j];
-            ri[j] = rb[row + n - U + j];
+            const long long pos = n - U + j;  // <= t
+            xi[j] = pos == t ? xv : xb[row + pos];
+            ri[j] = pos == t ? rv : rb[row + pos];
         }
 #pragma unroll
         for (int k = 1; k < 2 * U; ++k) {
-            xp[k] = xb[row + k];
-            rp[k] = rb[row + k];
+            // positions above t are still zero (the power-of-two case reads them)
+            xp[k] = k == t ? xv : xb[row + k];
+            rp[k] = k == t ? rv : rb[row + k];
         }
+#pragma unroll
+        for (int r = 0; r < U; ++r) ao[r] = acc[row + n + r];
+    }
+    y_t[g] = t == 0 ? rv * xv : fmaf(r0, xv, fmaf(rv, x0, run));
+    xb[row + t] = xv;
+    rb[row + t] = rv;
+    if (U > 0) {
+        const bool both = (n & (n - 1)) != 0;
 #pragma unroll
         for (int r = 0; r < U; ++r) {
             float s = 0.f;
@@ -62,7 +67,7 @@ __global__ void k_dd_step(float* __restrict__ xb, float* __restrict__ rb, float*
                 s = fmaf(xi[j], rp[U + r - j], s);
                 if (both) s = fmaf(ri[j], xp[U + r - j], s);
             }
-            acc[row + n + r] += s;
+            acc[row + n + r] = ao[r] + s;
         }
     }
 }
