@@ -1059,21 +1059,30 @@ int choose_window(fi_ctx* c) {
     return FI_OK;  // W = 0: window path unavailable, per-token path only
 }
 
+// Device time of one launch of the blocks released at n with implementation impl:
+// one warm-up launch, then `reps` launches each between its own pair of events; the
+// median (robust to a launch that met a clock or scheduling hiccup).
 float time_launch(fi_ctx* c, long long n, int impl, int reps) {
-    cudaEvent_t e0, e1;
-    cudaEventCreate(&e0);
-    cudaEventCreate(&e1);
     if (launch_block(c, n, impl, c->cap)) return -1.f;
-    cudaEventRecord(e0, c->cap);
-    for (int r = 0; r < reps; ++r)
-        if (launch_block(c, n, impl, c->cap)) return -1.f;
-    cudaEventRecord(e1, c->cap);
-    cudaEventSynchronize(e1);
-    float ms = 0.f;
-    cudaEventElapsedTime(&ms, e0, e1);
-    cudaEventDestroy(e0);
-    cudaEventDestroy(e1);
-    return ms * 1000.f / reps;
+    std::vector<cudaEvent_t> ev(reps + 1);
+    for (auto& e : ev) cudaEventCreate(&e);
+    bool ok = cudaEventRecord(ev[0], c->cap) == cudaSuccess;
+    for (int r = 0; r < reps && ok; ++r) {
+        if (launch_block(c, n, impl, c->cap)) ok = false;
+        if (ok) ok = cudaEventRecord(ev[r + 1], c->cap) == cudaSuccess;
+    }
+    std::vector<float> us;
+    if (ok && cudaEventSynchronize(ev[reps]) == cudaSuccess) {
+        for (int r = 0; r < reps; ++r) {
+            float ms = 0.f;
+            cudaEventElapsedTime(&ms, ev[r], ev[r + 1]);
+            us.push_back(1000.f * ms);
+        }
+    }
+    for (auto& e : ev) cudaEventDestroy(e);
+    if (us.size() != (size_t)reps) return -1.f;
+    std::sort(us.begin(), us.end());
+    return us[reps / 2];
 }
 
 // Hybrid tau: time each implementation able to serve block size 2^q and keep the
@@ -1087,8 +1096,8 @@ int autotune(fi_ctx* c) {
         const bool can_f = c->spec[q] != nullptr;
         float td = 0.f, tf = 0.f;
         if (can_d && can_f) {
-            td = time_launch(c, U, FI_TAU_DIRECT, 3);
-            tf = time_launch(c, U, FI_TAU_FFT, 3);
+            td = time_launch(c, U, FI_TAU_DIRECT, 7);
+            tf = time_launch(c, U, FI_TAU_FFT, 7);
             if (td < 0 || tf < 0) return FI_ECUDA;
         }
         c->tau_us[q][0] = td;
