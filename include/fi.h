@@ -330,8 +330,10 @@ int fi_lm_split(fi_lm *m, double *mixer_us, double *total_us);
  * Layout: x, rho and the running sums are [G][L] float32 on the device. */
 typedef struct fi_dd fi_dd;
 
-/* G >= 1 channels; L a power of two, 2 <= L <= 2^17.  Device memory: 3 G L floats plus
- * about 2.5 G L complex values of spectra.  Returns NULL on error (fi_last_error). */
+/* G >= 1 channels; L a power of two, 2 <= L <= 2^17.  Device memory: 3 G L floats (x,
+ * rho, running sums) plus about 1.5 G L complex values of spectra (both prefixes for
+ * every block size up to L/4, and the power-of-two block's up to L/2).  Returns NULL
+ * on error (fi_last_error). */
 fi_dd *fi_dd_create(int G, int L);
 
 /* Release the context.  NULL is accepted. */
