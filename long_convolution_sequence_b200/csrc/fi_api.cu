@@ -2127,7 +2127,8 @@ int fi_lm_split(fi_lm* m, double* mixer_us, double* total_us) {
 // ---------------------------------------------------------------- data-dependent filter
 // The long convolution with a filter that arrives online with the data (fi.h,
 // fi_dd_create): red cells per step (k_dd_step, which also adds the blocks of U <= 8
-// on the direct tau), then the larger blocks released after the step's token: two of the same size U = lowbit(n) at a step n that is not a power of
+// on the direct tau; k_dd_window for a whole aligned window given at once), then the
+// larger blocks released after the step's token: two of the same size U = lowbit(n) at a step n that is not a power of
 // two (x against rho's prefix, rho against x's prefix), one at n = U (x against rho
 // with its unknown tail still zero).  The FFT form uses the spectra of the prefixes
 // x[0, 2U) and rho[0, 2U), made at step 2U; the power-of-two block uses the spectrum
@@ -2192,19 +2193,58 @@ int dd_block(fi_dd* d, long long n, bool x_input, const float2* spec, cudaStream
     return launch_fft(q, a, st);
 }
 
+// The blocks released after the n-th token (n < L): two of size U = lowbit(n), or at a
+// power of two one, preceded by the spectra that become final there.
+int dd_release(fi_dd* d, long long n, cudaStream_t st) {
+    const int G = d->G;
+    const long long L = d->L;
+    const int q = ctz64(n);
+    int rc;
+    if (is_pow2(n)) {
+        // the prefixes of length n are final: spectra for the blocks of size n / 2
+        // still to come (steps 3n/2, 5n/2, ...)
+        if (q >= 1) {
+            const int q2 = q - 1;
+            if (dd_tau(d, q2) == FI_TAU_FFT && (3LL << q2) < L) {
+                if ((rc = make_spectra(q2, d->xb, L, G, d->spx[q2], d->c->tw, st))) return rc;
+                if ((rc = make_spectra(q2, d->rb, L, G, d->spr[q2], d->c->tw, st))) return rc;
+            }
+        }
+        if (dd_tau(d, q) == FI_TAU_FFT && (rc = make_spectra(q, d->rb, L, G, d->spz, d->c->tw, st))) return rc;
+        return dd_block(d, n, true, d->spz, st);
+    }
+    if ((rc = dd_block(d, n, true, d->spr[q], st))) return rc;
+    return dd_block(d, n, false, d->spx[q], st);
+}
+
+// Steps d->t .. d->t + steps - 1.  A whole aligned window of kDdWin steps at kW >= kDdWin
+// runs as one k_dd_window launch (the blocks of U < kDdWin inside it folded in), then
+// the blocks released at its end; every other step runs on its own (k_dd_step, with
+// the blocks of U <= 8 inside it), then its larger blocks.
 int dd_run(fi_dd* d, const float* x, const float* rho, int steps, float* y, cudaStream_t st) {
     const int G = d->G;
     const long long L = d->L;
+    constexpr int W = kDdWin;
     int rc;
-    for (int k = 0; k < steps; ++k) {
-        const long long t = d->t + k;
+    const long long t0 = d->t, t_end = d->t + steps;
+    long long t = t0;
+    while (t < t_end) {
+        const size_t k = (size_t)(t - t0);
+        const float *xk = x + k * G, *rk = rho + k * G;
+        float* yk = y + k * G;
+        if (t >= W && t % W == 0 && t + W <= t_end) {
+            k_dd_window<W><<<(G + kDdWinCh - 1) / kDdWinCh, 256, dd_window_smem<W>(), st>>>(d->xb, d->rb, d->acc, xk,
+                                                                                          rk, yk, t, G, L);
+            CK(cudaGetLastError());
+            if (t + W < L && (rc = dd_release(d, t + W, st))) return rc;
+            t += W;
+            continue;
+        }
         const long long n = t + 1;
         const int q = n < L ? ctz64(n) : -1;
         // blocks of U <= 8 on the direct tau run inside the step kernel
         const int fused = (q >= 0 && q <= 3 && dd_tau(d, q) == FI_TAU_DIRECT) ? (1 << q) : 0;
         const dim3 grid((G + 127) / 128), blk(128);
-        const float *xk = x + (size_t)k * G, *rk = rho + (size_t)k * G;
-        float* yk = y + (size_t)k * G;
         switch (fused) {
             case 1: k_dd_step<1><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
             case 2: k_dd_step<2><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
@@ -2213,23 +2253,8 @@ int dd_run(fi_dd* d, const float* x, const float* rho, int steps, float* y, cuda
             default: k_dd_step<0><<<grid, blk, 0, st>>>(d->xb, d->rb, d->acc, xk, rk, yk, t, G, L); break;
         }
         CK(cudaGetLastError());
-        if (n >= L || fused) continue;
-        if (is_pow2(n)) {
-            // the prefixes of length n are final: spectra for the blocks of size n / 2
-            // still to come (steps 3n/2, 5n/2, ...)
-            if (q >= 1) {
-                const int q2 = q - 1;
-                if (dd_tau(d, q2) == FI_TAU_FFT && (3LL << q2) < L) {
-                    if ((rc = make_spectra(q2, d->xb, L, G, d->spx[q2], d->c->tw, st))) return rc;
-                    if ((rc = make_spectra(q2, d->rb, L, G, d->spr[q2], d->c->tw, st))) return rc;
-                }
-            }
-            if (dd_tau(d, q) == FI_TAU_FFT && (rc = make_spectra(q, d->rb, L, G, d->spz, d->c->tw, st))) return rc;
-            if ((rc = dd_block(d, n, true, d->spz, st))) return rc;
-        } else {
-            if ((rc = dd_block(d, n, true, d->spr[q], st))) return rc;
-            if ((rc = dd_block(d, n, false, d->spx[q], st))) return rc;
-        }
+        if (n < L && !fused && (rc = dd_release(d, n, st))) return rc;
+        ++t;
     }
     return FI_OK;
 }
@@ -2254,6 +2279,8 @@ void dd_free(fi_dd* d) {
 int dd_create_impl(fi_dd* d) {
     int rc = set_all_attrs();
     if (rc) return rc;
+    CK(cudaFuncSetAttribute(k_dd_window<kDdWin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            (int)dd_window_smem<kDdWin>()));
     fi_ctx* c = new fi_ctx();
     d->c = c;
     CK(cudaGetDevice(&c->dev));

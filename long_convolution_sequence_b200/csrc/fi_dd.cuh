@@ -72,4 +72,85 @@ __global__ void k_dd_step(float* __restrict__ xb, float* __restrict__ rb, float*
     }
 }
 
+// A whole aligned window [kW, kW + W) of steps at once, kW >= W, when its inputs are
+// all given.  The blocks of size U < W released inside the window read and write only
+// the window (Algorithm 1's window property), and together they add, for every pair of
+// window positions j < t, x_j rho_{t-j} + rho_j x_{t-j}: the window's values against
+// the prefixes' first W values (lags t - j < W <= kW, so the lag indices are prefix
+// indices and never window ones).  With the running sums staged (the blocks released at
+// or before kW), every output of the window is then
+//   y_t = acc[t] + rho_0 x_t + rho_t x_0 + sum_{j=kW}^{t-1} (x_j rho_{t-j} + rho_j x_{t-j}),
+// independent of the window's other outputs: no step has to wait for another.  The
+// in-window blocks are not added to the running sums (they would only feed positions
+// of this window, all final here).  One CTA: 32 channels x W steps; inputs x_in, rho_in
+// and outputs y_out are [W][G] rows of the caller's arrays; x and rho also go to their
+// [G][L] buffers for the blocks of U >= W.  Shared memory rows are padded to W + 1
+// floats, so that the 32 channels of a warp (one step) read 32 different banks.
+constexpr int kDdWinCh = 32;
+constexpr int kDdWin = 128;
+template <int W>
+constexpr size_t dd_window_smem() { return sizeof(float) * 4 * kDdWinCh * (W + 1); }
+
+template <int W>
+__global__ void __launch_bounds__(256) k_dd_window(float* __restrict__ xb, float* __restrict__ rb,
+                                                   const float* __restrict__ acc, const float* __restrict__ x_in,
+                                                   const float* __restrict__ rho_in, float* __restrict__ y_out,
+                                                   long long kW, int G, long long L) {
+    constexpr int NT = 256, P = W + 1, C = kDdWinCh;
+    extern __shared__ float dd_sm[];  // [4][C][W + 1]
+    float(*sx)[P] = reinterpret_cast<float(*)[P]>(dd_sm);
+    float(*sr)[P] = reinterpret_cast<float(*)[P]>(dd_sm + C * P);
+    float(*px)[P] = reinterpret_cast<float(*)[P]>(dd_sm + 2 * C * P);
+    float(*pr)[P] = reinterpret_cast<float(*)[P]>(dd_sm + 3 * C * P);
+    const int g0 = blockIdx.x * C;
+    const int nc = min(C, G - g0);
+    const int tid = threadIdx.x;
+    // the window's inputs, [W][G] rows: 32 channels of one step per warp (128 bytes)
+    for (int e = tid; e < W * C; e += NT) {
+        const int s = e / C, c = e - s * C;
+        float xv = 0.f, rv = 0.f;
+        if (c < nc) {
+            xv = x_in[(long long)s * G + g0 + c];
+            rv = rho_in[(long long)s * G + g0 + c];
+        }
+        sx[c][s] = xv;
+        sr[c][s] = rv;
+    }
+    // the prefixes' first W values of every channel (positions 0 .. W-1 < kW)
+    for (int e = tid; e < W * C; e += NT) {
+        const int c = e / W, k = e - c * W;
+        float xv = 0.f, rv = 0.f;
+        if (c < nc) {
+            xv = xb[(long long)(g0 + c) * L + k];
+            rv = rb[(long long)(g0 + c) * L + k];
+        }
+        px[c][k] = xv;
+        pr[c][k] = rv;
+    }
+    __syncthreads();
+    // the window's values into the [G][L] buffers (row segments of W floats)
+    for (int e = tid; e < W * C; e += NT) {
+        const int c = e / W, k = e - c * W;
+        if (c < nc) {
+            xb[(long long)(g0 + c) * L + kW + k] = sx[c][k];
+            rb[(long long)(g0 + c) * L + kW + k] = sr[c][k];
+        }
+    }
+    // outputs: thread (c, j) takes the steps s = j, j + 8, ... of channel c
+    const int c = tid % C, j = tid / C;
+    constexpr int NJ = NT / C;
+    for (int s = j; s < W; s += NJ) {
+        float v = 0.f;
+        if (c < nc) {
+            const long long row = (long long)(g0 + c) * L;
+            const float a = acc[row + kW + s];
+            float sum = 0.f;
+            for (int lag = 1; lag <= s; ++lag)
+                sum = fmaf(sx[c][s - lag], pr[c][lag], fmaf(sr[c][s - lag], px[c][lag], sum));
+            v = fmaf(pr[c][0], sx[c][s], fmaf(sr[c][s], px[c][0], a + sum));
+        }
+        if (c < nc) y_out[(long long)s * G + g0 + c] = v;
+    }
+}
+
 }  // namespace fi
