@@ -343,8 +343,10 @@ void fi_dd_destroy(fi_dd *d);
 int fi_dd_reset(fi_dd *d);
 
 /* Steps t .. t+steps-1: x and rho [steps][G] float32 (host or device) are the inputs of
- * those steps; y [steps][G] (host or device) receives the outputs.  FI_ECAPACITY past
- * L; FI_EINVAL for a NULL array with steps > 0. */
+ * those steps; y [steps][G] (host or device, not overlapping x or rho) receives the
+ * outputs.  Each aligned window of 128 steps at or after step 128 that the call covers
+ * whole is evaluated in one launch (its inputs are all given); other steps one at a
+ * time.  FI_ECAPACITY past L; FI_EINVAL for a NULL array with steps > 0. */
 int fi_dd_forward(fi_dd *d, const float *x, const float *rho, int steps, float *y);
 
 /* The implementation of blocks of size 2^q: FI_TAU_DIRECT (q <= 12), FI_TAU_FFT
