@@ -84,3 +84,63 @@ def test_delta_filter_and_delta_input():
     y = dd.run(x, d3)
     np.testing.assert_array_equal(y[3:], x[:-3])
     np.testing.assert_array_equal(y[:3], 0.0)
+
+
+# ----------------------------------------------------------------- the pins can fail
+# Each plausible mistake is planted in a copy of oracle/dd.py's source (loaded as a
+# module of its own; the oracle itself is untouched) and must break at least one pin.
+DD_MUTANTS = {
+    "mirror_block_at_powers_of_two": ("        if not is_pow2(n):\n            out.append((n, \"rho\", U))",
+                                      "        out.append((n, \"rho\", U))"),
+    "reads_unknown_tail": ("            if is_pow2(n) and lag >= U:\n                continue           # rho[U, 2U)",
+                           "            if False:\n                continue           # rho[U, 2U)"),
+    "run_reads_unknown_tail": ("                    if is_pow2(n) and lag >= U:\n                        continue",
+                               "                    if False:\n                        continue"),
+    "run_lag_off_by_one": ("                    lag = n + r - s\n", "                    lag = n + r - s - 1\n"),
+    "run_drops_red_cell": ("            y[t] += rb[t] * xb[0]", "            y[t] += 0.0"),
+    "run_mirror_at_powers_of_two": ("            if kind == \"rho\" and is_pow2(n):\n                continue",
+                                    "            if False:\n                continue"),
+}
+
+
+def _planted(name):
+    import importlib.util
+    import sys
+    import types
+    from pathlib import Path
+    src = Path(dd.__file__).read_text()
+    old, new = DD_MUTANTS[name]
+    assert src.count(old) == 1, name
+    mod = types.ModuleType("dd_mutant_" + name)
+    exec(compile(src.replace(old, new), "dd_mutant_" + name, "exec"), mod.__dict__)
+    return mod
+
+
+def _pins_pass(mod):
+    """True if every pin above holds for the module `mod` standing in for oracle.dd."""
+    global dd
+    real = dd
+    dd = mod
+    try:
+        for L in (8, 33, 64):
+            test_every_product_added_exactly_once_when_both_factors_are_known(L)
+        for P in (4, 8):
+            test_two_convolutions_of_the_same_size_per_step(P)
+        for T, G in ((37, 4), (130, 2)):
+            test_online_evaluation_is_the_causal_convolution(T, G)
+        test_roles_of_input_and_filter_are_symmetric()
+        test_delta_filter_and_delta_input()
+        return True
+    except AssertionError:
+        return False
+    finally:
+        dd = real
+
+
+def test_the_unmodified_oracle_passes_the_pins():
+    assert _pins_pass(dd)
+
+
+@pytest.mark.parametrize("name", sorted(DD_MUTANTS))
+def test_every_planted_mistake_fails_a_pin(name):
+    assert not _pins_pass(_planted(name)), name
