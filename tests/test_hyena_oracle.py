@@ -125,3 +125,61 @@ def test_one_layer_with_a_delta_filter_against_torch():
         u2 = r + bf(T.nn.functional.gelu(bf(ln(r)) @ W1.T)) @ W2.T
         np.testing.assert_allclose(out["u"][t], u2.numpy(), rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(out["logits"][t], (bf(ln(u2)) @ Wlm.T).numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- the pins can fail
+# Each plausible mistake is planted in a copy of oracle/hyena.py's source (loaded as a
+# module of its own; the oracle itself is untouched) and must break at least one pin.
+HYENA_MUTANTS = {
+    "gemv_operand_not_rounded": ("    return bf16_round(a) @ np.asarray(W, dtype=np.float64).T",
+                                 "    return np.asarray(a, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T"),
+    "short_conv_wrong_tap": ("c[1] * z_hist[1] + c[2] * z_hist[2]", "c[1] * z_hist[2] + c[2] * z_hist[1]"),
+    "layer_norm_without_eps": ("    return (x - mu) / np.sqrt(var + LN_EPS)", "    return (x - mu) / np.sqrt(var)"),
+    "gelu_tanh_form": ("    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))",
+                       "    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))"),
+    "gate_uses_q": ("            x_hist[l, t] = k * v", "            x_hist[l, t] = q * v"),
+    "residual_dropped": ("            u = r + m", "            u = m"),
+    "mixer_lag_off_by_one": ("            lag = h[l][:, t::-1][:, : t + 1]",
+                             "            lag = np.concatenate([h[l][:, t + 1:t + 2], h[l][:, t::-1]], axis=1)[:, : t + 1]"),
+    "output_gate_dropped": ("            r = u + q * y", "            r = u + y"),
+}
+
+
+def _planted(name):
+    import types
+    from pathlib import Path
+    src = Path(hyena.__file__).read_text()
+    old, new = HYENA_MUTANTS[name]
+    assert src.count(old) == 1, name
+    mod = types.ModuleType("hyena_mutant_" + name)
+    exec(compile(src.replace(old, new), "hyena_mutant_" + name, "exec"), mod.__dict__)
+    return mod
+
+
+def _pins_pass(mod):
+    """True if every pin above holds with `mod` standing in for oracle.hyena."""
+    global hyena
+    real = hyena
+    hyena = mod
+    try:
+        test_bf16_round_matches_torch_including_ties()
+        test_layer_norm_and_gelu_match_torch()
+        test_short_conv_closed_forms()
+        test_the_long_convolution_inside_the_model_is_the_causal_convolution()
+        test_identity_layers_reduce_to_embedding_and_lm_head()
+        test_teacher_forced_and_closed_loop_agree_on_the_closed_loops_tokens()
+        test_one_layer_with_a_delta_filter_against_torch()
+        return True
+    except AssertionError:
+        return False
+    finally:
+        hyena = real
+
+
+def test_the_unmodified_oracle_passes_the_pins():
+    assert _pins_pass(hyena)
+
+
+@pytest.mark.parametrize("name", sorted(HYENA_MUTANTS))
+def test_every_planted_mistake_fails_a_pin(name):
+    assert not _pins_pass(_planted(name)), name
