@@ -700,6 +700,19 @@ def bench_ablation(args):
 LM_CONFIG = dict(M=18, B=4, D=768, L=1 << 15, V=50257)
 
 
+def lm_model_bytes(M, B, D, L, V):
+    """Algorithmic bytes of one greedy generation of L tokens: per token the bf16
+    weights each GEMV streams (W_in 3D x D, W1 4D x D, W2 D x 4D per layer, the LM head
+    V x D) and the embedding rows (B x D), 2 bytes each; the mixers' blocks, 20U bytes
+    per block and chain (4U(3B'+2) at one row per chain) over M x B x D chains, one block
+    of U = lowbit(n) after token n; and per token and chain of every layer the mixer
+    step's state (the short-convolution ring, the input and running sum, 40 bytes)."""
+    weights = (M * (3 * D * D + 4 * D * D + 4 * D * D) + V * D + B * D) * 2
+    G = B * D
+    blocks = sum(20 * (n & -n) for n in range(1, L)) * M * G
+    return L * weights + blocks + L * M * G * 40
+
+
 def bench_lm(args):
     """The Hyena-like model end to end (BASELINE configuration 5): greedy generation of
     L tokens from uniform random start tokens, random-init weights (bf16 GEMMs, fp32
@@ -781,6 +794,12 @@ def bench_lm(args):
     lm.close()
     rms = float(np.sqrt(np.mean(ref["logits"] ** 2)))
     logit_err = float(np.abs(lg - ref["logits"]).max()) / rms
+    hbm, src, _ = peaks()
+    nbytes = lm_model_bytes(M, B, D, L, V)
+    ach = nbytes / (ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+            "traffic": None, "kernel": "whole generation", "model_bytes": nbytes,
+            "peak_source": src + " (MEASURED_PEAKS.json hbm_gbs)"}
     line = {"metric": "end-to-end tokens/s (B*L/time), Hyena-like model, greedy decoding", "value": round(B * L / (ms / 1e3), 1),
             "unit": "tokens/s", "ms_per_generation": round(ms, 1), "steps": steps, "dtype": "bf16 GEMMs / f32 mixer",
             "data": "synthetic: random-init weights, uniform random start tokens",
@@ -792,6 +811,7 @@ def bench_lm(args):
                                     "every 64th token (scaled)"},
             "host_issue_ms": round(host_ms, 1),
             "graphs_off": {"ms_per_generation": round(ms_eager, 1), "host_issue_ms": round(host_ms_eager, 1)},
+            "roofline": roof,
             "oracle_check": {"tokens": T_s, "max_logit_err_over_rms": logit_err,
                              "bound": (3 * M + 1) * 2.0 ** -8,
                              "greedy_agree": int((tf == ref["next"]).sum()), "of": int(tf.size)},
