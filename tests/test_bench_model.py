@@ -52,3 +52,19 @@ def test_sweep_memory_model():
     # the sweep's largest point does not fit one B200, the headline does
     assert bench.sweep_need_bytes(18, 8, 1024, 1 << 18) > 180e9
     assert bench.sweep_need_bytes(18, 1, 864, 1 << 17) < 100e9
+
+
+def test_data_dependent_bytes_follow_the_oracles_schedule():
+    # 20U bytes per block of the data-dependent tiling (one at powers of two, two
+    # elsewhere: oracle.dd.schedule) plus 24 per red cell, per channel
+    from oracle import dd
+    for G, L in ((1, 16), (3, 256), (7, 1 << 12)):
+        want = G * (sum(20 * U for _, _, U in dd.schedule(L)) + 24 * L)
+        assert bench.dd_model_bytes(G, L) == want
+
+
+def test_language_model_bytes_by_hand():
+    # one layer, B = 1, D = 8, L = 4, V = 10: per token 2 (3*64 + 4*64 + 4*64 + 10*8 + 8)
+    # = 1584 bytes; blocks after tokens 1, 2, 3 (U = 1, 2, 1) at 20U per chain over 8
+    # chains = 640; mixer state 40 per chain and token = 1280
+    assert bench.lm_model_bytes(1, 1, 8, 4, 10) == 4 * 1584 + 640 + 1280
