@@ -136,20 +136,50 @@ __global__ void __launch_bounds__(256) k_dd_window(float* __restrict__ xb, float
             rb[(long long)(g0 + c) * L + kW + k] = sr[c][k];
         }
     }
-    // outputs: thread (c, j) takes the steps s = j, j + 8, ... of channel c
-    const int c = tid % C, j = tid / C;
-    constexpr int NJ = NT / C;
-    for (int s = j; s < W; s += NJ) {
-        float v = 0.f;
-        if (c < nc) {
-            const long long row = (long long)(g0 + c) * L;
-            const float a = acc[row + kW + s];
-            float sum = 0.f;
-            for (int lag = 1; lag <= s; ++lag)
-                sum = fmaf(sx[c][s - lag], pr[c][lag], fmaf(sr[c][s - lag], px[c][lag], sum));
-            v = fmaf(pr[c][0], sx[c][s], fmaf(sr[c][s], px[c][0], a + sum));
+    // outputs: thread (c, jb) takes two blocks of 8 consecutive steps of channel c, jb and
+    // 15 - jb (their triangles together as long as any other pair).  Per chunk of 8 lags
+    // it holds the 15 window values of each sequence those lags reach and the 8 prefix
+    // values: 46 shared-memory reads per 128 multiply-adds.  A lag past the row (only
+    // beyond every step of the block, where the window value is taken as zero) is
+    // clamped to the row's last entry.
+    constexpr int QB = 8, NB = W / QB;
+    static_assert(NT / C * 2 == NB, "two blocks of 8 steps per thread cover the window");
+    const int c = tid % C, jb = tid / C;
+    if (c < nc) {
+        const long long row = (long long)(g0 + c) * L;
+        const float x0 = px[c][0], r0 = pr[c][0];
+        for (int half = 0; half < 2; ++half) {
+            const int s0 = (half == 0 ? jb : NB - 1 - jb) * QB;
+            float accq[QB];
+#pragma unroll
+            for (int q = 0; q < QB; ++q) accq[q] = 0.f;
+            for (int l0 = 1; l0 <= s0 + QB - 1; l0 += 8) {
+                float xv[QB + 7], rv[QB + 7], pl[8], xl[8];
+#pragma unroll
+                for (int m = 0; m < QB + 7; ++m) {
+                    const int pos = s0 - l0 - 7 + m;  // window position s0 + q - (l0 + d), m = q - d + 7
+                    xv[m] = pos >= 0 ? sx[c][pos] : 0.f;
+                    rv[m] = pos >= 0 ? sr[c][pos] : 0.f;
+                }
+#pragma unroll
+                for (int d = 0; d < 8; ++d) {
+                    const int lg = min(l0 + d, W - 1);
+                    pl[d] = pr[c][lg];
+                    xl[d] = px[c][lg];
+                }
+#pragma unroll
+                for (int d = 0; d < 8; ++d)
+#pragma unroll
+                    for (int q = 0; q < QB; ++q)
+                        accq[q] = fmaf(xv[q - d + 7], pl[d], fmaf(rv[q - d + 7], xl[d], accq[q]));
+            }
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+                const int s = s0 + q;
+                const float v = fmaf(r0, sx[c][s], fmaf(sr[c][s], x0, acc[row + kW + s] + accq[q]));
+                y_out[(long long)s * G + g0 + c] = v;
+            }
         }
-        if (c < nc) y_out[(long long)s * G + g0 + c] = v;
     }
 }
 
