@@ -214,11 +214,14 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
     // operands for the first step are loaded now, in the shadow of the staging
     long long t = ep.t;
     MixOps mo;
-    const bool mix_lane = MIX && lane < B && (KS == 1 || warp % KS == 0);
+    // (the owner of value (q, b) of the reduce-scatter below: lane b << SHM)
+    constexpr int SHM = RPW * BM <= 4 ? 3 : RPW * BM <= 8 ? 2 : RPW * BM <= 16 ? 1 : 0;
+    const int mix_b = lane >> SHM;
+    const bool mix_lane = MIX && (lane & ((1 << SHM) - 1)) == 0 && mix_b < B && (KS == 1 || warp % KS == 0);
     if (MIX) {
         if (ep.io) t = ep.io->t;
         const int d = blockIdx.x * UPC + warp / KS;
-        if (mix_lane && d < NU) mo = lm_mixer_load(lane, d, ep.zr, ep.conv, ep.h, ep.L, B, ep.D, t, ep.Y, x);
+        if (mix_lane && d < NU) mo = lm_mixer_load(mix_b, d, ep.zr, ep.conv, ep.h, ep.L, B, ep.D, t, ep.Y, x);
     }
     {
         // the inputs into the two planes, twelve 16-byte loads a thread in flight at once
@@ -338,25 +341,36 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
                 }
             }
         }
-        // sums over the lanes (every lane ends with all of them)
+        // sums over the lanes as a reduce-scatter: value v = r BM + b (RPW BM of them,
+        // padded to NP, a power of two); at the level of offset 2^k a lane keeps the half
+        // of its values that bit k of its id selects and adds its partner's copy of it,
+        // until one value is left (v = lane >> SH); the lanes that share it then add
+        // across the remaining low bits.  NP - 1 + SH shuffles instead of 5 per value.
+        constexpr int NP = RPW * BM <= 4 ? 4 : RPW * BM <= 8 ? 8 : RPW * BM <= 16 ? 16 : 32;
+        constexpr int SH = NP == 4 ? 3 : NP == 8 ? 2 : NP == 16 ? 1 : 0;
+        float vals[NP];
 #pragma unroll
-        for (int r = 0; r < RPW; ++r)
+        for (int v = 0; v < NP; ++v) vals[v] = v < RPW * BM ? acc[v / BM][v % BM] : 0.f;
 #pragma unroll
-            for (int b = 0; b < BM; ++b)
-                if (b < B) {
+        for (int k = 4; k >= SH; --k) {
+            const int half = 1 << (k - SH);
+            const bool up = (lane >> k) & 1;
 #pragma unroll
-                    for (int o = 16; o; o >>= 1) acc[r][b] += __shfl_xor_sync(0xffffffffu, acc[r][b], o);
-                }
-        // lane (rl, bl) = (lane / BM, lane % BM) finishes row rl of the step for batch row
-        // bl; with KS > 1 the writing warp adds the partial sums of the warps sharing its rows
-        const int rl = lane / BM, bl = lane % BM;
-        float a = 0.f;
+            for (int i = 0; i < half; ++i) {
+                const float send = up ? vals[i] : vals[i + half];
+                const float keep = up ? vals[i + half] : vals[i];
+                vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << k);
+            }
+        }
+        float a = vals[0];
 #pragma unroll
-        for (int r = 0; r < RPW; ++r)
-#pragma unroll
-            for (int b = 0; b < BM; ++b)
-                if (r == rl && b == bl) a = acc[r][b];
-        const bool pair = rl < RPW && bl < B;
+        for (int o = (1 << SH) >> 1; o >= 1; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        // the lane with low bits zero owns value v = lane >> SH: row rl = v / BM of the
+        // step, batch row bl = v % BM; with KS > 1 the writing warp adds the partial sums
+        // of the warps sharing its rows
+        const int v = lane >> SH;
+        const int rl = v / BM, bl = v % BM;
+        const bool pair = (lane & ((1 << SH) - 1)) == 0 && rl < RPW && bl < B;
         if (KS > 1) {
             if (pair) part[warp][rl][bl] = a;
             __syncthreads();
@@ -367,14 +381,14 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
             __syncthreads();
         }
         if (MIX) {
-            // lane (0, b) gathers k and v of batch row b from lanes (1, b), (2, b)
-            const float zk = __shfl_sync(0xffffffffu, a, (lane + BM) & 31);
-            const float zv = __shfl_sync(0xffffffffu, a, (lane + 2 * BM) & 31);
+            // the owner of (q, b) gathers k and v of batch row b from the owners of (k, b), (v, b)
+            const float zk = __shfl_sync(0xffffffffu, a, (lane + (BM << SH)) & 31);
+            const float zv = __shfl_sync(0xffffffffu, a, (lane + (2 * BM << SH)) & 31);
             const int d = u0 + warp / KS;
             if (mix_lane && d < NU) {
                 if (u0 != blockIdx.x * UPC)
-                    mo = lm_mixer_load(lane, d, ep.zr, ep.conv, ep.h, ep.L, B, ep.D, t, ep.Y, x);
-                lm_mixer_finish(mo, a, zk, zv, lane, d, ep.zr, ep.L, B, ep.D, t, ep.X, ep.Y, y);
+                    mo = lm_mixer_load(mix_b, d, ep.zr, ep.conv, ep.h, ep.L, B, ep.D, t, ep.Y, x);
+                lm_mixer_finish(mo, a, zk, zv, mix_b, d, ep.zr, ep.L, B, ep.D, t, ep.X, ep.Y, y);
             }
             continue;
         }
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(kLmThreads, kLmCtasPerSm) k_lm_gemv(const __nv
             // the step's best per batch row: a maximum over the lanes of equal bl
             unsigned long long k = own ? lm_key(a, n) : 0ull;
 #pragma unroll
-            for (int o = BM; o < RPW * BM; o <<= 1) {
+            for (int o = BM << SH; o < (RPW * BM) << SH; o <<= 1) {
                 const unsigned long long q = __shfl_xor_sync(0xffffffffu, k, o);
                 k = q > k ? q : k;
             }
