@@ -46,12 +46,13 @@ __device__ __forceinline__ int lm_key_id(unsigned long long k) { return (int)(0x
 
 // u[b][:] = E[tok[b]][:] (bf16 embedding rows to fp32)
 //
-// The kernels are written to run under programmatic dependent launch (they read
-// nothing their predecessors write before griddepcontrol.wait, and the matrix-vector
-// kernels prefetch their weight rows into L2 before it), but the host launches them
-// without it: releasing each successor at once made the launches cascade and the
-// waiting CTAs crowd the running kernel.  Reads of data another kernel writes go
-// through L2 only (ld.global.cg), which stays correct however the launches overlap.
+// The kernels run under programmatic dependent launch: they read nothing their
+// predecessors write before griddepcontrol.wait (the matrix-vector kernels prefetch
+// their weight rows into L2 and issue their first weight loads before it), and each
+// releases its successor only once its own wait has returned, so at most one launch
+// waits behind the running one (releasing successors at kernel start made the
+// launches cascade).  Reads of data another kernel writes go through L2 only
+// (ld.global.cg), which stays correct however the launches overlap.
 __global__ void k_lm_embed(const __nv_bfloat16* __restrict__ E, const int* __restrict__ tok, int B, int D,
                            float* __restrict__ u, unsigned long long* amax) {
     grid_dep_wait();
