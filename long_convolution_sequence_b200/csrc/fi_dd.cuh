@@ -1,8 +1,10 @@
 // fi_dd.cuh -- device code of the long convolution with a data-dependent filter
-// (sm_100a): the red cells of one step.  The blocks are the tile kernels of
-// fi_kernels.cuh (direct or FFT tau) with one layer of G channels: Algorithm 1's block
-// with the input sequence's buffer as `act`, the other sequence's buffer as the taps
-// `h`, and the running sums as `act_out`.
+// (sm_100a): one step's red cells with its blocks of U <= 8 (k_dd_step), and a whole
+// aligned window of given steps with every block below the window's size folded in
+// (k_dd_window).  The larger blocks are the tile kernels of fi_kernels.cuh (direct or
+// FFT tau) with one layer of G channels: Algorithm 1's block with the input sequence's
+// buffer as `act`, the other sequence's buffer as the taps `h`, and the running sums
+// as `act_out`.
 //
 // The Flash Inference summary (section "Technische Innovationen", item 4,
 // "Datenabhaengige Filter-Erweiterung") and the rebuttal's answer on data-dependent
